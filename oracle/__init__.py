@@ -1,0 +1,260 @@
+"""CPU oracle for the FP8 quantize / scaling-aware direct transpose path.
+
+TEST INFRASTRUCTURE.  Only the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product library
+(``scaling_aware_transpose_b200``) never imports, links or calls it, and it shares no
+code with it: the C source here is an independent, plain restatement of the method's
+definitions (see the header of ``fp8q_oracle.c`` for the passages each function
+follows).
+
+Arrays are numpy: bf16 tensors travel as ``uint16`` bit patterns, FP8 codes and UE8M0
+scale bytes as ``uint8``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = ctypes.CDLL(path)
+        _declare(_lib)
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _declare(L):
+    V, I64, I32, D, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_float
+    L.orc_e4m3_encode.argtypes, L.orc_e4m3_encode.restype = [D], ctypes.c_uint8
+    L.orc_e4m3_decode.argtypes, L.orc_e4m3_decode.restype = [ctypes.c_uint8], D
+    L.orc_scale_exponent.argtypes, L.orc_scale_exponent.restype = [D], ctypes.c_int
+    L.orc_shift_code_value.argtypes = [ctypes.c_uint8, ctypes.c_int]
+    L.orc_shift_code_value.restype = ctypes.c_uint8
+    L.orc_shift_code_bytes.argtypes = [ctypes.c_uint8, ctypes.c_int]
+    L.orc_shift_code_bytes.restype = ctypes.c_uint8
+    for name, args in {
+        "orc_e4m3_encode_array": [V, I64, V],
+        "orc_e4m3_decode_array": [V, I64, V],
+        "orc_scale_exponent_array": [V, I64, V],
+        "orc_shift_codes": [V, I64, ctypes.c_int, ctypes.c_int, V],
+        "orc_quantize_rowwise": [V, I64, I64, V, V],
+        "orc_quantize_rowwise_f32": [V, I64, I64, V, V],
+        "orc_exp_spec_constants": [V],
+        "orc_exp_spec_array": [V, I64, V],
+        "orc_swiglu_array": [V, V, I64, V],
+    }.items():
+        fn = getattr(L, name)
+        fn.argtypes, fn.restype = args, None
+    for name, args in {
+        "orc_direct_transpose": [V, V, I64, I64, V, I32, V, V],
+        "orc_naive_transpose": [V, V, I64, I64, V, I32, V, V],
+        "orc_swiglu_quant": [V, V, I64, I64, V, V, V, V],
+        "orc_permute_pad_quant": [V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
+    }.items():
+        fn = getattr(L, name)
+        fn.argtypes, fn.restype = args, ctypes.c_int
+    L.orc_exp_spec.argtypes, L.orc_exp_spec.restype = [F], F
+    L.orc_num_threads.argtypes, L.orc_num_threads.restype = [], ctypes.c_int
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---------------------------------------------------------------- codec
+def e4m3_encode(y) -> np.ndarray:
+    y = _c(y, np.float64)
+    out = np.empty(y.shape, np.uint8)
+    lib().orc_e4m3_encode_array(_p(y), y.size, _p(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    c = _c(c, np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib().orc_e4m3_decode_array(_p(c), c.size, _p(out))
+    return out
+
+
+def scale_exponent(amax) -> np.ndarray:
+    a = _c(amax, np.float64)
+    out = np.empty(a.shape, np.int32)
+    lib().orc_scale_exponent_array(_p(a), a.size, _p(out))
+    return out
+
+
+def shift_codes(codes, k: int, rule: str = "value") -> np.ndarray:
+    c = _c(codes, np.uint8)
+    out = np.empty(c.shape, np.uint8)
+    lib().orc_shift_codes(_p(c), c.size, int(k), 1 if rule == "bytes" else 0, _p(out))
+    return out
+
+
+# ---------------------------------------------------------------- path steps
+def quantize_rowwise(x_bf16_bits):
+    x = _c(x_bf16_bits, np.uint16)
+    rows, cols = x.shape
+    if cols % 128:
+        raise OracleError("cols must be a multiple of 128")
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // 128), np.uint8)
+    lib().orc_quantize_rowwise(_p(x), rows, cols, _p(q), _p(sf))
+    return q, sf
+
+
+def quantize_rowwise_f32(y):
+    y = _c(y, np.float32)
+    rows, cols = y.shape
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // 128), np.uint8)
+    lib().orc_quantize_rowwise_f32(_p(y), rows, cols, _p(q), _p(sf))
+    return q, sf
+
+
+def _transpose_common(fn, q, sf, offsets):
+    q = _c(q, np.uint8)
+    sf = _c(sf, np.uint8)
+    rows, cols = q.shape
+    off = None if offsets is None else _c(offsets, np.int32)
+    G = 1 if off is None else off.size - 1
+    qt = np.zeros(rows * cols, np.uint8)
+    sft = np.zeros(rows * cols // 128, np.uint8)
+    rc = fn(_p(q), _p(sf), rows, cols, _p(off), G, _p(qt), _p(sft))
+    if rc:
+        raise OracleError(f"oracle transpose rejected its arguments (code {rc})")
+    if off is None:
+        return qt.reshape(cols, rows), sft.reshape(cols, rows // 128)
+    return qt, sft  # flat: group g at cols*off[g], shape [cols, M_g]
+
+
+def direct_transpose(q, sf, offsets=None):
+    """Dense: returns (Q^T [cols, rows], SF^T [cols, rows/128]).  Grouped (offsets):
+    returns the flat output buffers, group g at cols*off_g with shape [cols, M_g]."""
+    return _transpose_common(lib().orc_direct_transpose, q, sf, offsets)
+
+
+def naive_transpose(q, sf, offsets=None):
+    return _transpose_common(lib().orc_naive_transpose, q, sf, offsets)
+
+
+def exp_spec(a) -> np.ndarray:
+    a = _c(a, np.float32)
+    out = np.empty(a.shape, np.float32)
+    lib().orc_exp_spec_array(_p(a), a.size, _p(out))
+    return out
+
+
+def exp_spec_constants() -> np.ndarray:
+    out = np.empty(11, np.float32)
+    lib().orc_exp_spec_constants(_p(out))
+    return out
+
+
+def swiglu(g, u) -> np.ndarray:
+    g = _c(g, np.float32)
+    u = _c(u, np.float32)
+    out = np.empty(g.shape, np.float32)
+    lib().orc_swiglu_array(_p(g), _p(u), g.size, _p(out))
+    return out
+
+
+def swiglu_quant(gate_bits, up_bits, transposed: bool = True):
+    g = _c(gate_bits, np.uint16)
+    u = _c(up_bits, np.uint16)
+    rows, cols = g.shape
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // 128), np.uint8)
+    qt = np.empty((cols, rows), np.uint8) if transposed else None
+    sft = np.empty((cols, rows // 128), np.uint8) if transposed else None
+    rc = lib().orc_swiglu_quant(_p(g), _p(u), rows, cols, _p(q), _p(sf), _p(qt), _p(sft))
+    if rc:
+        raise OracleError(f"oracle swiglu_quant rejected its arguments (code {rc})")
+    return q, sf, qt, sft
+
+
+def permute_max_rows(tokens: int, topk: int, num_experts: int, align: int) -> int:
+    return tokens * topk + num_experts * (align - 1)
+
+
+def permute_pad_quant(x_bits, topk_idx, num_experts: int, align: int, max_rows: int | None = None,
+                      fill: int = 0xEE):
+    """Returns (Q [max_rows, H], SF [max_rows, H/128], offsets [E+1], row_id_map [T*K]).
+    Rows at or beyond offsets[E] keep the `fill` byte (they are not written)."""
+    x = _c(x_bits, np.uint16)
+    idx = _c(topk_idx, np.int32)
+    T, H = x.shape
+    K = idx.shape[1] if idx.ndim == 2 else 1
+    if max_rows is None:
+        max_rows = permute_max_rows(T, K, num_experts, align)
+    q = np.full((max_rows, H), fill, np.uint8)
+    sf = np.full((max_rows, H // 128), fill, np.uint8)
+    off = np.zeros(num_experts + 1, np.int32)
+    rmap = np.zeros(T * K, np.int32)
+    rc = lib().orc_permute_pad_quant(_p(x), T, H, _p(idx), K, num_experts, align, _p(q), _p(sf),
+                                     max_rows, _p(off), _p(rmap))
+    if rc:
+        raise OracleError(f"oracle permute_pad_quant rejected its arguments (code {rc})")
+    return q, sf, off, rmap
+
+
+def num_threads() -> int:
+    return int(lib().orc_num_threads())
+
+
+# ---------------------------------------------------------------- error report
+# Reported numbers, not parity: how far each column-wise result lands from the
+# original tensor (the "double quantization error" of the FP8-Flow-MoE review,
+# section 问题与动机), and DeepGEMM's calc_diff (DeepSeek FP8 与 DeepGEMM, §5.7).
+
+def dequant_rowwise(q, sf) -> np.ndarray:
+    vals = e4m3_decode(q)
+    e = sf.astype(np.int64) - 127
+    return vals * np.exp2(np.repeat(e, 128, axis=1).astype(np.float64))
+
+
+def dequant_colwise(qt, sft) -> np.ndarray:
+    """Dense Q^T [cols, rows] + SF^T [cols, rows/128] -> values [rows, cols]."""
+    return dequant_rowwise(qt, sft).T
+
+
+def naive_fp32_colwise(v: np.ndarray) -> np.ndarray:
+    """Column requantization with non-power-of-two fp32 scales amax/448 (the SM90
+    DeepGEMM convention, DeepSeek FP8 与 DeepGEMM §3): report-only reference for the
+    genuine double-quantization case.  v: [rows, cols] float64, rows % 128 == 0.
+    Returns the dequantized column-wise values [rows, cols]."""
+    rows, cols = v.shape
+    t = v.reshape(rows // 128, 128, cols)
+    amax = np.abs(t).max(axis=1, keepdims=True).astype(np.float32)
+    s = np.where(amax > 0, (amax / np.float32(448.0)).astype(np.float32), np.float32(1.0)).astype(np.float64)
+    codes = e4m3_encode(t / s)
+    return (e4m3_decode(codes) * s).reshape(rows, cols)
+
+
+def rel_rms(approx: np.ndarray, exact: np.ndarray) -> float:
+    exact = np.asarray(exact, np.float64)
+    num = np.sqrt(np.sum((np.asarray(approx, np.float64) - exact) ** 2))
+    den = np.sqrt(np.sum(exact ** 2))
+    return float(num / den) if den > 0 else 0.0
+
+
+def calc_diff(x: np.ndarray, y: np.ndarray) -> float:
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    den = np.sum(x * x + y * y)
+    return float(1.0 - 2.0 * np.sum(x * y) / den) if den > 0 else 0.0

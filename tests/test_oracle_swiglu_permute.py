@@ -1,0 +1,153 @@
+"""Pins for the oracle's fused SwiGLU+quantize (FP8-Flow-MoE review, 核心方法: Fused
+SwiGLU+Quantization) and fused permute+pad+quantize (核心方法: Fused Permute+Padding;
+DeepSeek FP8 与 DeepGEMM §5.6: experts' rows concatenated along M)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from scaling_aware_transpose_b200 import synthetic
+
+
+def ulp_distance_f32(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    ia = a.astype(np.float32).view(np.int32).astype(np.int64)
+    ib = b.astype(np.float32).view(np.int32).astype(np.int64)
+    ia = np.where(ia < 0, -(ia & 0x7FFFFFFF), ia)
+    ib = np.where(ib < 0, -(ib & 0x7FFFFFFF), ib)
+    return np.abs(ia - ib)
+
+
+def test_exp_spec_constants_are_derived():
+    c = oracle.exp_spec_constants()
+    ln2 = math.log(2.0)
+    hi = np.float32(np.frombuffer(np.uint32(0x3F317200).tobytes(), np.float32)[0])
+    assert c[0] == np.float32(math.log2(math.e))
+    assert c[1] == hi and abs(float(hi) - ln2) < 2e-6
+    assert c[2] == np.float32(ln2 - float(hi))
+    for k in range(8):
+        assert c[3 + k] == np.float32(1.0 / math.factorial(k))
+
+
+def test_exp_spec_accuracy_vs_libm():
+    """Within 2 ulp of exp over the normal-result range, measured against exp in
+    double rounded once to fp32."""
+    rng = np.random.default_rng(8)
+    a = np.concatenate([rng.uniform(-87.0, 88.5, 400000), rng.uniform(-1, 1, 100000),
+                        np.linspace(-87, 88.5, 100001)]).astype(np.float32)
+    got = oracle.exp_spec(a)
+    ref = np.exp(a.astype(np.float64)).astype(np.float32)
+    d = ulp_distance_f32(got, ref)
+    assert d.max() <= 2, float(d.max())
+
+
+def test_exp_spec_special_values():
+    a = np.array([0.0, 89.5, 1e30, -104.5, -1e30, 88.0, -103.0], np.float32)
+    e = oracle.exp_spec(a)
+    assert e[0] == 1.0 and np.isinf(e[1]) and np.isinf(e[2])
+    assert e[3] == 0.0 and e[4] == 0.0
+    assert np.isfinite(e[5]) and e[6] > 0  # subnormal, not flushed
+
+
+def test_swiglu_special_values():
+    g = np.array([0.0, 30.0, -200.0, 1.0, -1.0], np.float32)
+    u = np.array([5.0, 2.0, 3.0, 1.0, 1.0], np.float32)
+    y = oracle.swiglu(g, u)
+    assert y[0] == 0.0
+    assert y[1] == np.float32(60.0)  # silu(30) rounds to 30 in fp32
+    assert y[2] == 0.0 and np.signbit(y[2])
+    ref = np.array([1.0 / (1.0 + math.exp(-1.0)), -1.0 / (1.0 + math.exp(1.0))])
+    assert np.allclose(y[3:], ref, rtol=3e-7)
+
+
+def test_swiglu_close_to_double_reference():
+    rng = np.random.default_rng(9)
+    g = rng.standard_normal(200000).astype(np.float32) * 4
+    u = rng.standard_normal(200000).astype(np.float32)
+    y = oracle.swiglu(g, u).astype(np.float64)
+    gd, ud = g.astype(np.float64), u.astype(np.float64)
+    ref = gd / (1.0 + np.exp(-gd)) * ud
+    assert np.all(np.abs(y - ref) <= 4 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64) + 1e-45)
+
+
+def test_swiglu_quant_is_quantize_of_swiglu_then_direct():
+    d = synthetic.swiglu(rows=256, cols=384, seed=10)
+    q, sf, qt, sft = oracle.swiglu_quant(d["gate"], d["up"])
+    g = synthetic.bf16_bits_to_f32(d["gate"])
+    u = synthetic.bf16_bits_to_f32(d["up"])
+    y = oracle.swiglu(g, u)
+    rq, rsf = oracle.quantize_rowwise_f32(y)
+    assert np.array_equal(q, rq) and np.array_equal(sf, rsf)
+    dqt, dsft = oracle.direct_transpose(q, sf)
+    assert np.array_equal(qt, dqt) and np.array_equal(sft, dsft)
+    q2, sf2, qt2, sft2 = oracle.swiglu_quant(d["gate"], d["up"], transposed=False)
+    assert qt2 is None and np.array_equal(q2, q)
+
+
+# ------------------------------------------------------------------ permute
+
+def brute_permute(x_bits, idx, E, align):
+    T, K = idx.shape
+    H = x_bits.shape[1]
+    pairs = {e: [] for e in range(E)}
+    for t in range(T):
+        for s in range(K):
+            pairs[int(idx[t, s])].append((t, s))
+    off = [0]
+    for e in range(E):
+        n = len(pairs[e])
+        off.append(off[-1] + (n + align - 1) // align * align)
+    rmap = np.zeros(T * K, np.int32)
+    for e in range(E):
+        for r, (t, s) in enumerate(pairs[e]):
+            rmap[t * K + s] = off[e] + r
+    qx, sfx = oracle.quantize_rowwise(x_bits)
+    q = np.full((off[-1], H), 0xEE, np.uint8)
+    sf = np.full((off[-1], H // 128), 0xEE, np.uint8)
+    for p in range(T * K):
+        q[rmap[p]], sf[rmap[p]] = qx[p // K], sfx[p // K]
+    for e in range(E):
+        for r in range(off[e] + len(pairs[e]), off[e + 1]):
+            q[r], sf[r] = 0, 127
+    return q, sf, np.array(off, np.int32), rmap
+
+
+@pytest.mark.parametrize("align", [1, 2, 16])
+def test_permute_brute_force_tiny(align):
+    rng = np.random.default_rng(11 + align)
+    T, E, K, H = 8, 4, 2, 256
+    x = synthetic.scaled_normal(T, H, seed=12)
+    idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    q, sf, off, rmap = oracle.permute_pad_quant(x, idx, E, align)
+    bq, bsf, boff, brmap = brute_permute(x, idx, E, align)
+    n = boff[-1]
+    assert np.array_equal(off, boff) and np.array_equal(rmap, brmap)
+    assert np.array_equal(q[:n], bq) and np.array_equal(sf[:n], bsf)
+    assert np.all(q[n:] == 0xEE) and np.all(sf[n:] == 0xEE)
+
+
+def test_permute_invariants_zipf():
+    d = synthetic.moe(tokens=512, hidden=256, num_experts=32, topk=8, seed=13)
+    align = 128
+    q, sf, off, rmap = oracle.permute_pad_quant(d["x"], d["topk_idx"], 32, align)
+    idx = d["topk_idx"]
+    counts = np.bincount(idx.ravel(), minlength=32)
+    assert counts.sum() == 512 * 8
+    sizes = np.diff(off)
+    assert np.all(sizes % align == 0) and np.all(sizes >= counts) and np.all(sizes - counts < align)
+    assert len(np.unique(rmap)) == rmap.size
+    e_of = idx.ravel()
+    assert np.all((rmap >= off[e_of]) & (rmap < off[e_of] + counts[e_of]))
+    # stable order: within an expert the rows follow (token, slot) order
+    for e in range(32):
+        r = rmap[e_of == e]
+        assert np.all(np.diff(r) == 1)
+    qx, sfx = oracle.quantize_rowwise(d["x"])
+    assert np.array_equal(q[rmap], np.repeat(qx, 8, axis=0))
+    assert np.array_equal(sf[rmap], np.repeat(sfx, 8, axis=0))
+
+
+def test_permute_rejects_bad_index():
+    x = synthetic.scaled_normal(4, 128, seed=14)
+    with pytest.raises(oracle.OracleError):
+        oracle.permute_pad_quant(x, np.array([[0], [1], [5], [2]], np.int32), 4, 16)
