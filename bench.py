@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 quantize + scaling-aware direct transpose hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch of the dense-activation workload
+(X bf16 [8192, 7168], N(0,1) times a lognormal(0, 1.5) row factor, 7 outlier channels
+x100): fp8q_quantize_rowwise (X -> Q, SF) then fp8q_direct_transpose (Q, SF -> Q^T, SF^T).
+Each kernel is timed with CUDA events on the launching stream after an L2 flush (a
+256 MiB device write, outside the events), so both read their inputs from HBM.  The
+metric is algorithmic HBM bytes / kernel time (every input byte read once, every output
+byte written once), in GB/s.  With N ranks (torchrun, one GPU each) every rank runs its
+own batch (weak scaling, no collective on the data path); the value is all ranks' bytes
+over the slowest rank's time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (plain C, the parity reference) on the host cores
+on a bounded sample of the same workload; only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "dense activation X bf16 [8192, 7168]: N(0,1) x lognormal(0,1.5) per row, 7 outlier channels x100"
+ROWS, COLS = 8192, 7168
+N_ELEM = ROWS * COLS
+BYTES_QUANT = 2 * N_ELEM + N_ELEM + N_ELEM // 128            # read X, write Q + SF
+BYTES_DIRECT = N_ELEM + N_ELEM // 128 + N_ELEM + N_ELEM // 128  # read Q + SF, write Q^T + SF^T
+BYTES_STEP = BYTES_QUANT + BYTES_DIRECT
+METRIC = "direct-transpose & quantize GB/s on 1 B200 (% of HBM peak); bit-exact vs oracle"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ host helpers
+def measured_peak_gbs():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources(kind: str):
+    csrc = os.path.join(ROOT, "scaling_aware_transpose_b200", "csrc")
+    main = {"quantize": "quantize_rowwise.cu", "direct": "direct_transpose.cu"}[kind]
+    return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")]
+
+
+def source_digest(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kind: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on this
+    workload, or None when there is none or the kernel source changed since."""
+    name = {"quantize": "quantize_rowwise_dense_8192x7168.md", "direct": "direct_transpose_dense_8192x7168.md"}[kind]
+    p = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"dram_bytes_per_launch:\s*(\d+)", txt)
+    s = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
+    if not m or not s or s.group(1) != source_digest(kernel_sources(kind)):
+        return None
+    return int(m.group(1))
+
+
+def roofline(bytes_per_launch: int, avg_seconds: float, peak_gbs: float, peak_kind: str, traffic):
+    achieved = bytes_per_launch / avg_seconds / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak_gbs, "unit": "GB/s",
+            "frac": round(achieved / peak_gbs, 4), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_kind == "measured" else "fallback", "traffic": traffic}
+
+
+def reduce_max(value: float, dist_mod=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist_mod is None or not dist_mod.is_initialized() or dist_mod.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event (throttle) reasons through NVML in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period, self.idx, self._stop, self._t = period_s, device_index, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        reasons = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml" if self._nv else "unavailable"}
+
+
+def cpu_baseline(x_bits, budget_s: float = 10.0, max_reps: int = 50):
+    """The oracle (quantize + direct transpose) as it stands, on the host cores, over the
+    full workload, repeated until the time budget is spent."""
+    import oracle
+    times, reps = [], 0
+    t_end = time.perf_counter() + budget_s
+    while reps < max_reps and (reps < 1 or time.perf_counter() < t_end):
+        t0 = time.perf_counter()
+        q, sf = oracle.quantize_rowwise(x_bits)
+        oracle.direct_transpose(q, sf)
+        times.append(time.perf_counter() - t0)
+        reps += 1
+    rows = x_bits.shape[0]
+    step_bytes = BYTES_STEP * rows // ROWS
+    avg = sum(times) / len(times)
+    return {"value": round(step_bytes / avg / 1e9, 3), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{rows}x{COLS} rows of the workload (quantize + direct transpose), "
+                                        f"{reps} repetitions, {sum(times):.1f} s"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import scaling_aware_transpose_b200 as sat
+    from scaling_aware_transpose_b200 import synthetic
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    sat.lib()  # fail loudly here if the library is missing
+    x_bits = synthetic.dense(seed=rank)["x"]
+    x_host = synthetic.to_torch_bf16(x_bits).pin_memory()
+    x = x_host.to(device)
+    q = torch.empty((ROWS, COLS), dtype=torch.uint8, device=device)
+    sf = torch.empty((ROWS, COLS // 128), dtype=torch.uint8, device=device)
+    qt = torch.empty((COLS, ROWS), dtype=torch.uint8, device=device)
+    sft = torch.empty((COLS, ROWS // 128), dtype=torch.uint8, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+
+    def quant():
+        sat.fp8q_quantize_rowwise(x, ROWS, COLS, q, sf, sp)
+
+    def direct():
+        sat.fp8q_direct_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, sp)
+
+    def step(evs=None):
+        flush.fill_(1)
+        if evs:
+            evs[0].record(stream)
+        quant()
+        if evs:
+            evs[1].record(stream)
+        flush.fill_(2)
+        if evs:
+            evs[2].record(stream)
+        direct()
+        if evs:
+            evs[3].record(stream)
+
+    W = max(3, args.warmup)
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if sat.fp8q_last_device_status(sp) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for k in range(K):
+            step(evs[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    tq = [e[0].elapsed_time(e[1]) * 1e-3 for e in evs]
+    td = [e[2].elapsed_time(e[3]) * 1e-3 for e in evs]
+    total = sum(tq) + sum(td)
+    total_max = reduce_max(total, dist, device)
+    status = sat.fp8q_last_device_status(sp)
+    if status != 0:
+        raise RuntimeError(f"device status {sat.STATUS.get(status)} after the timed region")
+
+    # ---- extra, untimed-by-the-headline measurements
+    # back-to-back step (no flush between the two kernels: Q stays in L2)
+    chained = []
+    for _ in range(min(K, 50)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(3)
+        a.record(stream)
+        quant()
+        direct()
+        b.record(stream)
+        chained.append((a, b))
+    # naive three-pass path on the same Q, SF
+    ws = torch.empty(sat.fp8q_naive_workspace_bytes(ROWS, COLS), dtype=torch.uint8, device=device)
+    nqt, nsft = torch.empty_like(qt), torch.empty_like(sft)
+    naive = []
+    for i in range(min(K, 50) + 3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(4)
+        a.record(stream)
+        sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, nqt, nsft, ws, ws.numel(), sp)
+        b.record(stream)
+        if i >= 3:
+            naive.append((a, b))
+    torch.cuda.synchronize()
+    t_chain = statistics.median(a.elapsed_time(b) * 1e-3 for a, b in chained)
+    t_naive = statistics.median(a.elapsed_time(b) * 1e-3 for a, b in naive)
+
+    # ---- end to end through the C ABI from pinned host buffers
+    q_h = torch.empty_like(q, device="cpu").pin_memory()
+    sf_h = torch.empty_like(sf, device="cpu").pin_memory()
+    qt_h = torch.empty_like(qt, device="cpu").pin_memory()
+    sft_h = torch.empty_like(sft, device="cpu").pin_memory()
+    e2e = []
+    for i in range(min(K, 20) + 2):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x.copy_(x_host, non_blocking=True)
+        quant()
+        direct()
+        q_h.copy_(q, non_blocking=True)
+        sf_h.copy_(sf, non_blocking=True)
+        qt_h.copy_(qt, non_blocking=True)
+        sft_h.copy_(sft, non_blocking=True)
+        b.record(stream)
+        if i >= 2:
+            e2e.append((a, b))
+    torch.cuda.synchronize()
+    t_e2e = reduce_max(sum(a.elapsed_time(b) * 1e-3 for a, b in e2e) / len(e2e), dist, device)
+    ok_e2e = bool(np.array_equal(qt_h.numpy(), qt.cpu().numpy()))
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peak_gbs()
+    avg_q, avg_d = sum(tq) / K, sum(td) / K
+    dominant = "quantize" if avg_q >= avg_d else "direct"
+    rf = roofline(BYTES_QUANT if dominant == "quantize" else BYTES_DIRECT, max(avg_q, avg_d), peak, peak_kind,
+                  profiled_traffic(dominant))
+    rf["kernel"] = {"quantize": "fp8q_quantize_rowwise (quantize_tiles_kernel)",
+                    "direct": "fp8q_direct_transpose (direct_transpose_kernel)"}[dominant]
+    value = world * K * BYTES_STEP / total_max / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(total_max / K * 1e3, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "path": "fp8q_quantize_rowwise -> fp8q_direct_transpose",
+                   "bytes_per_step": BYTES_STEP, "l2": "flushed before each kernel (256 MiB device write, "
+                   "outside the events)", "seed": "rank", "parallelism": f"replicas x{world} (no collective)"},
+        "roofline": rf,
+        "kernels": {
+            "quantize_rowwise": {"us": round(avg_q * 1e6, 2), "GB/s": round(BYTES_QUANT / avg_q / 1e9, 1),
+                                 "frac_of_peak": round(BYTES_QUANT / avg_q / 1e9 / peak, 4),
+                                 "frac_of_8000": round(BYTES_QUANT / avg_q / 1e9 / 8000, 4),
+                                 "traffic": profiled_traffic("quantize")},
+            "direct_transpose": {"us": round(avg_d * 1e6, 2), "GB/s": round(BYTES_DIRECT / avg_d / 1e9, 1),
+                                 "frac_of_peak": round(BYTES_DIRECT / avg_d / 1e9 / peak, 4),
+                                 "frac_of_8000": round(BYTES_DIRECT / avg_d / 1e9 / 8000, 4),
+                                 "traffic": profiled_traffic("direct")},
+            "naive_transpose_3pass": {"us": round(t_naive * 1e6, 2),
+                                      "GB/s_of_direct_bytes": round(BYTES_DIRECT / t_naive / 1e9, 1),
+                                      "direct_speedup": round(t_naive / avg_d, 2)},
+            "chained_step_no_flush_between": {"us": round(t_chain * 1e6, 2),
+                                              "GB/s": round(BYTES_STEP / t_chain / 1e9, 1)},
+        },
+        "gpu_launches": 2 * K,
+        "e2e": {"value": round(BYTES_STEP / t_e2e / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": 2 * N_ELEM,
+                "d2h_bytes_per_step": 2 * N_ELEM + 2 * (N_ELEM // 128), "ms_per_step": round(t_e2e * 1e3, 3),
+                "result_matches_device": ok_e2e},
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x_bits, budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    import oracle
+    from scaling_aware_transpose_b200 import synthetic
+    x_bits = synthetic.dense(seed=0)["x"][: args.ref_rows]
+    rows = x_bits.shape[0]
+    W = max(3, args.warmup)
+    for _ in range(W):
+        q, sf = oracle.quantize_rowwise(x_bits)
+        oracle.direct_transpose(q, sf)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        q, sf = oracle.quantize_rowwise(x_bits)
+        oracle.direct_transpose(q, sf)
+    total = time.perf_counter() - t0
+    step_bytes = BYTES_STEP * rows // ROWS
+    value = args.steps * step_bytes / total / 1e9
+    sample = f"{rows}x{COLS} rows of the workload per step (quantize + direct transpose)"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": W, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "path": "CPU oracle: quantize_rowwise -> direct_transpose",
+                   "bytes_per_step": step_bytes, "sample": sample},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
+    args = ap.parse_args(argv)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1:
+        import torch
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,169 @@
+/*
+ * fp8q.h — C ABI of libfp8q: the FP8 data-movement hot path of FP8-Flow-MoE on one
+ * B200 (sm_100a).
+ *
+ *   row-wise 1x128 E4M3 quantization with power-of-two (UE8M0) scales
+ *   -> scaling-aware direct transpose to the column-wise (1x128 along tokens) layout,
+ * plus the in-library naive dequant->transpose->requant baseline and the fused
+ * SwiGLU+quantize and permute+pad+quantize neighbours.
+ *
+ * Sources (page title, section):
+ *   "FP8-Flow-MoE: A Casting-Free FP8 Recipe without Double Quantization Error
+ *    (MLSys 2026)" review: 核心方法 (scaling-aware transpose; fused permute+padding;
+ *    fused SwiGLU+quantization), 关键观察 2, 问题与动机 (the naive three-pass path).
+ *   "01 · DeepSeek FP8 与 DeepGEMM：Hopper 软件方案": §1 (wgrad reduces over tokens),
+ *    §3 (1x128 activation tiles, SF [T, C/128], online amax), §5.6 (M-grouped
+ *    contiguous expert layout), §8 (UE8M0 scales).
+ *   "低精度（Low Precision）：从 FP8 到 FP4 的训练与推理" §2 (E4M3: max 448, no Inf).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers on the current CUDA device, allocated and owned by
+ *     the caller; the library never allocates, frees or retains them.  Each must be
+ *     16-byte aligned and address a contiguous row-major array.
+ *   - E4M3 codes are bytes (OCP E4M3FN: bias 7, max 448, no Inf).  Scales are UE8M0
+ *     bytes: S = 2^(byte - 127).  An all-zero tile has scale byte 127 (S = 1).
+ *   - Each call is asynchronous on `stream` (NULL = the legacy default stream) and
+ *     returns after the launch.  Host-detectable argument errors return before any
+ *     launch and leave every output untouched.  Errors that only the device can see
+ *     (bad group offsets, routing indices out of range, a bounded wait that expired)
+ *     are recorded in one per-device status word; read it with
+ *     fp8q_last_device_status().
+ *   - Inputs must be finite (no NaN/Inf); codes given to the transposes must come from
+ *     a quantization (never 0x7F/0xFF).
+ *   - Calls that share an output buffer and overlap on the GPU race; order them on one
+ *     stream.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so that users need no CUDA header. */
+typedef struct CUstream_st *fp8q_stream_t;
+
+typedef enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_NULL = 1,    /* a required pointer is NULL */
+    FP8Q_ERR_SHAPE = 2,   /* sizes violate the layout rules (multiples of 128, groups) */
+    FP8Q_ERR_ALIGN = 3,   /* a pointer is not 16-byte aligned */
+    FP8Q_ERR_ARG = 4,     /* other invalid argument (workspace too small, capacity, ...) */
+    FP8Q_ERR_CUDA = 5,    /* a CUDA runtime/driver call failed (launch, attribute query) */
+    FP8Q_ERR_TIMEOUT = 6, /* device: a bounded wait on an mbarrier expired */
+    FP8Q_ERR_DEVICE = 7   /* device: invalid data seen by a kernel (e.g. expert index) */
+} fp8q_status;
+
+/* Static, NUL-terminated description of a status code. */
+const char *fp8q_status_string(fp8q_status s);
+
+/* Synchronizes `stream`, then reads and clears the current device's status word.
+ * Returns FP8Q_OK if no kernel recorded an error since the last read, the first
+ * recorded device error otherwise, or FP8Q_ERR_CUDA if the synchronization failed. */
+fp8q_status fp8q_last_device_status(fp8q_stream_t stream);
+
+/* Row-wise 1x128 quantization (DeepSeek FP8 §3; FP8-Flow-MoE 关键观察 2).
+ *   x  : bf16 [rows, cols], cols % 128 == 0, rows >= 0.
+ *   q  : u8   [rows, cols]      out: E4M3 codes, q = RNE(x / S) saturating at 448.
+ *   sf : u8   [rows, cols/128]  out: UE8M0 byte e + 127 of tile (t, j), where
+ *        e = ceil(log2(amax/448)) (the smallest e with amax <= 448 * 2^e), e = 0 for
+ *        an all-zero tile, clamped to [-127, 127].
+ * rows == 0 is a no-op.  Errors: NULL, ALIGN, SHAPE (cols % 128 != 0, negatives),
+ * CUDA. */
+fp8q_status fp8q_quantize_rowwise(const void *x, int64_t rows, int64_t cols, uint8_t *q, uint8_t *sf,
+                                  fp8q_stream_t stream);
+
+/* Scaling-aware direct transpose (FP8-Flow-MoE 核心方法).  For every 128x128 block
+ * (row block b, column block j): e_max = max of the block's 128 row-tile exponents;
+ * each row t shifts its codes by k_t = e_max - e_t >= 0, q' = RNE_e4m3(decode(q)*2^-k_t)
+ * (an exponent-field subtract, the mantissa re-rounded only when the result turns
+ * subnormal); the block is written transposed with scale byte e_max + 127 for each of
+ * its 128 channels.
+ *   q, sf : the row-wise pair from fp8q_quantize_rowwise, [rows, cols], [rows, cols/128].
+ *   group_offsets : NULL for one dense group (then rows % 128 == 0), or a DEVICE
+ *        int32 array [num_groups + 1] with offsets[0] == 0, non-decreasing, every
+ *        group size a multiple of 128, offsets[num_groups] <= rows (rows is then the
+ *        capacity of q).  Violations found on the device set FP8Q_ERR_SHAPE in the
+ *        status word and skip the offending blocks.
+ *   qt  : u8 out.  Dense: [cols, rows].  Grouped: group g (M_g = off[g+1]-off[g] rows)
+ *         is the row-major array [cols, M_g] starting at byte cols*off[g].
+ *   sft : u8 out.  Dense: [cols, rows/128].  Grouped: group g is [cols, M_g/128]
+ *         starting at byte cols*off[g]/128.
+ * Bytes past the last group are not written.  Errors: NULL, ALIGN, SHAPE, ARG
+ * (num_groups < 1), CUDA. */
+fp8q_status fp8q_direct_transpose(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t cols,
+                                  const int32_t *group_offsets, int32_t num_groups, uint8_t *qt,
+                                  uint8_t *sft, fp8q_stream_t stream);
+
+/* Bytes of device workspace fp8q_naive_transpose needs: 4 * rows * cols (a BF16
+ * dequantized copy and its BF16 transpose). */
+size_t fp8q_naive_workspace_bytes(int64_t rows, int64_t cols);
+
+/* Naive baseline that the direct transpose replaces (FP8-Flow-MoE 问题与动机 and
+ * 核心方法, the three-pass conversion): (1) dequantize each code to BF16,
+ * v = bf16(decode(q) * 2^e); (2) transpose v; (3) requantize every 128-token column
+ * tile with a fresh power-of-two scale by the rule of fp8q_quantize_rowwise.
+ * Three kernel launches.  Same arguments, layouts and errors as fp8q_direct_transpose,
+ * plus a caller-owned device workspace of at least fp8q_naive_workspace_bytes(rows,
+ * cols) bytes, 16-byte aligned (ERR_ARG if smaller). */
+fp8q_status fp8q_naive_transpose(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t cols,
+                                 const int32_t *group_offsets, int32_t num_groups, uint8_t *qt,
+                                 uint8_t *sft, void *workspace, size_t workspace_bytes,
+                                 fp8q_stream_t stream);
+
+/* Fused SwiGLU + quantization (FP8-Flow-MoE 核心方法: the activation is produced
+ * directly as FP8).  y = silu(gate) * up in fp32 with silu(g) = g / (1 + exp(-g)),
+ * every operation one IEEE fp32 rounding and exp the library's Cody-Waite/Taylor
+ * evaluation; then the row-wise quantization of y, and, if qt != NULL, the direct
+ * transpose of that result in the same kernel.
+ *   gate, up : bf16 [rows, cols], cols % 128 == 0.
+ *   q, sf    : out, as fp8q_quantize_rowwise.
+ *   qt, sft  : out, [cols, rows] and [cols, rows/128], or both NULL to skip; when given,
+ *              rows % 128 == 0.
+ * Errors: NULL, ALIGN, SHAPE, ARG (only one of qt/sft given), CUDA. */
+fp8q_status fp8q_swiglu_quant(const void *gate, const void *up, int64_t rows, int64_t cols, uint8_t *q,
+                              uint8_t *sf, uint8_t *qt, uint8_t *sft, fp8q_stream_t stream);
+
+/* Bytes of device workspace fp8q_permute_pad_quant needs. */
+size_t fp8q_permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts);
+
+/* Fused permute + pad + row-wise quantize (FP8-Flow-MoE 核心方法: Fused
+ * Permute+Padding; DeepSeek FP8 §5.6: M-grouped contiguous expert rows).
+ *   x        : bf16 [tokens, hidden], hidden % 128 == 0.
+ *   topk_idx : int32 [tokens, topk], expert ids in [0, num_experts).
+ *   Expert e receives the pairs (t, s) with topk_idx[t, s] == e, in (t, s) row-major
+ *   order; its segment is padded with zero rows to a multiple of `align`.
+ *   q, sf    : out [max_out_rows, hidden], [max_out_rows, hidden/128]; row r of the
+ *              segment of pair (t, s) holds the row-wise quantization of x[t]; padding
+ *              rows hold codes 0x00 and scale byte 127; rows at or beyond
+ *              expert_offsets[num_experts] are not written.
+ *   max_out_rows : capacity, >= tokens*topk + num_experts*(align-1).
+ *   expert_offsets : out int32 [num_experts + 1], exclusive scan of padded sizes.
+ *   row_id_map     : out int32 [tokens*topk], destination row of pair (t, s).
+ *   workspace      : device, >= fp8q_permute_workspace_bytes(...), 16-byte aligned.
+ *   align in [1, 4096]; num_experts in [1, 4096]; topk in [1, 64].
+ * An expert id out of range sets FP8Q_ERR_DEVICE in the status word (outputs are
+ * then unspecified).  Errors: NULL, ALIGN, SHAPE, ARG, CUDA. */
+fp8q_status fp8q_permute_pad_quant(const void *x, int64_t tokens, int64_t hidden, const int32_t *topk_idx,
+                                   int32_t topk, int32_t num_experts, int32_t align, uint8_t *q,
+                                   uint8_t *sf, int64_t max_out_rows, int32_t *expert_offsets,
+                                   int32_t *row_id_map, void *workspace, size_t workspace_bytes,
+                                   fp8q_stream_t stream);
+
+/* Test hook for the bounded-wait machinery (no counterpart on the pages): launches one
+ * CTA that waits on an mbarrier nobody arrives at, giving up after `timeout_ns`
+ * nanoseconds (clamped to [1e3, 2e9]); the kernel then records FP8Q_ERR_TIMEOUT in the
+ * status word and returns normally.  No fault, no trap: the context stays usable. */
+fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fp8q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -1,0 +1,235 @@
+"""scaling_aware_transpose_b200 — Python binding of libfp8q (the C ABI in include/fp8q.h).
+
+FP8-Flow-MoE's FP8 data-movement hot path on one B200: row-wise 1x128 E4M3
+quantization with power-of-two scales, the scaling-aware direct transpose to the
+column-wise layout, the naive three-pass baseline, fused SwiGLU+quantize and fused
+permute+pad+quantize.  Every step runs in the library's CUDA kernels; this module only
+marshals arguments (torch tensors -> device pointers, the current torch stream) and
+turns non-zero status codes into exceptions.  There is no CPU fallback: if libfp8q.so
+has not been built, every call raises.
+
+The functions named ``fp8q_*`` mirror the C entry points argument for argument;
+tensors stand in for pointers.  The lower-case helpers allocate outputs with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+
+STATUS = {
+    0: "FP8Q_OK", 1: "FP8Q_ERR_NULL", 2: "FP8Q_ERR_SHAPE", 3: "FP8Q_ERR_ALIGN", 4: "FP8Q_ERR_ARG",
+    5: "FP8Q_ERR_CUDA", 6: "FP8Q_ERR_TIMEOUT", 7: "FP8Q_ERR_DEVICE",
+}
+globals().update({name: code for code, name in STATUS.items()})
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)} ({_status_string(self.status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfp8q.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libfp8q.so is missing ({LIB_PATH}); build it with "
+                               "`python -m scaling_aware_transpose_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        sig = {
+            "fp8q_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "fp8q_last_device_status": ([P], ctypes.c_int),
+            "fp8q_quantize_rowwise": ([P, I64, I64, P, P, P], ctypes.c_int),
+            "fp8q_direct_transpose": ([P, P, I64, I64, P, I32, P, P, P], ctypes.c_int),
+            "fp8q_naive_workspace_bytes": ([I64, I64], SZ),
+            "fp8q_naive_transpose": ([P, P, I64, I64, P, I32, P, P, P, SZ, P], ctypes.c_int),
+            "fp8q_swiglu_quant": ([P, P, I64, I64, P, P, P, P, P], ctypes.c_int),
+            "fp8q_permute_workspace_bytes": ([I64, I32, I32], SZ),
+            "fp8q_permute_pad_quant": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
+            "fp8q_debug_expire_wait": ([ctypes.c_uint64, P], ctypes.c_int),
+            "fp8q_version": ([], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes, fn.restype = args, res
+        _lib = L
+    return _lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return lib().fp8q_status_string(int(code)).decode()
+    except Exception:  # pragma: no cover - only while reporting another error
+        return "?"
+
+
+# ---------------------------------------------------------------- marshalling
+def _ptr(t):
+    """Device pointer of a CUDA tensor (must be contiguous); ints pass through; None -> NULL."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libfp8q takes device tensors; got a tensor on " + str(t.device))
+    if not t.is_contiguous():
+        raise ValueError("libfp8q takes contiguous tensors")
+    return t.data_ptr() if t.numel() else None
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise Fp8qError(rc, where)
+
+
+# ---------------------------------------------------------------- C entry points
+def fp8q_last_device_status(stream=None) -> int:
+    return int(lib().fp8q_last_device_status(_stream(stream)))
+
+
+def fp8q_quantize_rowwise(x, rows: int, cols: int, q, sf, stream=None) -> None:
+    _check(lib().fp8q_quantize_rowwise(_ptr(x), rows, cols, _ptr(q), _ptr(sf), _stream(stream)),
+           "fp8q_quantize_rowwise")
+
+
+def fp8q_direct_transpose(q, sf, rows: int, cols: int, group_offsets, num_groups: int, qt, sft,
+                          stream=None) -> None:
+    _check(lib().fp8q_direct_transpose(_ptr(q), _ptr(sf), rows, cols, _ptr(group_offsets), num_groups,
+                                       _ptr(qt), _ptr(sft), _stream(stream)), "fp8q_direct_transpose")
+
+
+def fp8q_naive_workspace_bytes(rows: int, cols: int) -> int:
+    return int(lib().fp8q_naive_workspace_bytes(rows, cols))
+
+
+def fp8q_naive_transpose(q, sf, rows: int, cols: int, group_offsets, num_groups: int, qt, sft, workspace,
+                         workspace_bytes: int, stream=None) -> None:
+    _check(lib().fp8q_naive_transpose(_ptr(q), _ptr(sf), rows, cols, _ptr(group_offsets), num_groups,
+                                      _ptr(qt), _ptr(sft), _ptr(workspace), workspace_bytes,
+                                      _stream(stream)), "fp8q_naive_transpose")
+
+
+def fp8q_swiglu_quant(gate, up, rows: int, cols: int, q, sf, qt, sft, stream=None) -> None:
+    _check(lib().fp8q_swiglu_quant(_ptr(gate), _ptr(up), rows, cols, _ptr(q), _ptr(sf), _ptr(qt), _ptr(sft),
+                                   _stream(stream)), "fp8q_swiglu_quant")
+
+
+def fp8q_permute_workspace_bytes(tokens: int, topk: int, num_experts: int) -> int:
+    return int(lib().fp8q_permute_workspace_bytes(tokens, topk, num_experts))
+
+
+def fp8q_permute_pad_quant(x, tokens: int, hidden: int, topk_idx, topk: int, num_experts: int, align: int,
+                           q, sf, max_out_rows: int, expert_offsets, row_id_map, workspace,
+                           workspace_bytes: int, stream=None) -> None:
+    _check(lib().fp8q_permute_pad_quant(_ptr(x), tokens, hidden, _ptr(topk_idx), topk, num_experts, align,
+                                        _ptr(q), _ptr(sf), max_out_rows, _ptr(expert_offsets),
+                                        _ptr(row_id_map), _ptr(workspace), workspace_bytes,
+                                        _stream(stream)), "fp8q_permute_pad_quant")
+
+
+def fp8q_debug_expire_wait(timeout_ns: int, stream=None) -> None:
+    _check(lib().fp8q_debug_expire_wait(int(timeout_ns), _stream(stream)), "fp8q_debug_expire_wait")
+
+
+def fp8q_version() -> int:
+    return int(lib().fp8q_version())
+
+
+# ---------------------------------------------------------------- allocating helpers
+def _empty(shape, dtype, like):
+    import torch
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+def quantize_rowwise(x, stream=None):
+    """x: bf16 [rows, cols] on the GPU -> (q u8 [rows, cols], sf u8 [rows, cols/128])."""
+    import torch
+    rows, cols = x.shape
+    q = _empty((rows, cols), torch.uint8, x)
+    sf = _empty((rows, cols // 128), torch.uint8, x)
+    fp8q_quantize_rowwise(x, rows, cols, q, sf, stream)
+    return q, sf
+
+
+def direct_transpose(q, sf, group_offsets=None, stream=None):
+    """Dense: (Q^T [cols, rows], SF^T [cols, rows/128]).  Grouped (device int32 offsets):
+    flat buffers of rows*cols and rows*cols/128 bytes, group g at cols*off[g]."""
+    import torch
+    rows, cols = q.shape
+    G = 1 if group_offsets is None else group_offsets.numel() - 1
+    if group_offsets is None:
+        qt = _empty((cols, rows), torch.uint8, q)
+        sft = _empty((cols, rows // 128), torch.uint8, q)
+    else:
+        qt = _empty((rows * cols,), torch.uint8, q)
+        sft = _empty((rows * cols // 128,), torch.uint8, q)
+    fp8q_direct_transpose(q, sf, rows, cols, group_offsets, G, qt, sft, stream)
+    return qt, sft
+
+
+def naive_transpose(q, sf, group_offsets=None, workspace=None, stream=None):
+    import torch
+    rows, cols = q.shape
+    G = 1 if group_offsets is None else group_offsets.numel() - 1
+    need = fp8q_naive_workspace_bytes(rows, cols)
+    if workspace is None:
+        workspace = _empty((max(need, 16),), torch.uint8, q)
+    if group_offsets is None:
+        qt = _empty((cols, rows), torch.uint8, q)
+        sft = _empty((cols, rows // 128), torch.uint8, q)
+    else:
+        qt = _empty((rows * cols,), torch.uint8, q)
+        sft = _empty((rows * cols // 128,), torch.uint8, q)
+    fp8q_naive_transpose(q, sf, rows, cols, group_offsets, G, qt, sft, workspace, workspace.numel(), stream)
+    return qt, sft
+
+
+def swiglu_quant(gate, up, transposed: bool = True, stream=None):
+    import torch
+    rows, cols = gate.shape
+    q = _empty((rows, cols), torch.uint8, gate)
+    sf = _empty((rows, cols // 128), torch.uint8, gate)
+    qt = _empty((cols, rows), torch.uint8, gate) if transposed else None
+    sft = _empty((cols, rows // 128), torch.uint8, gate) if transposed else None
+    fp8q_swiglu_quant(gate, up, rows, cols, q, sf, qt, sft, stream)
+    return q, sf, qt, sft
+
+
+def permute_max_rows(tokens: int, topk: int, num_experts: int, align: int) -> int:
+    return tokens * topk + num_experts * (align - 1)
+
+
+def permute_pad_quant(x, topk_idx, num_experts: int, align: int, max_out_rows: int | None = None, stream=None):
+    """Returns (q [max_out_rows, H], sf [max_out_rows, H/128], expert_offsets [E+1],
+    row_id_map [T*K]); rows at or beyond expert_offsets[E] are left unwritten."""
+    import torch
+    tokens, hidden = x.shape
+    topk = topk_idx.shape[1]
+    if max_out_rows is None:
+        max_out_rows = permute_max_rows(tokens, topk, num_experts, align)
+    q = _empty((max_out_rows, hidden), torch.uint8, x)
+    sf = _empty((max_out_rows, hidden // 128), torch.uint8, x)
+    off = _empty((num_experts + 1,), torch.int32, x)
+    rmap = _empty((tokens * topk,), torch.int32, x)
+    ws_bytes = fp8q_permute_workspace_bytes(tokens, topk, num_experts)
+    ws = _empty((max(ws_bytes, 16),), torch.uint8, x)
+    fp8q_permute_pad_quant(x, tokens, hidden, topk_idx, topk, num_experts, align, q, sf, max_out_rows, off,
+                           rmap, ws, ws.numel(), stream)
+    return q, sf, off, rmap

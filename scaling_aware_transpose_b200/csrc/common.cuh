@@ -1,0 +1,215 @@
+// common.cuh — device helpers shared by the libfp8q kernels (sm_100a).
+//
+// E4M3 codes use the OCP E4M3FN layout (low-precision format table: 1/4/3 bits, max
+// 448, no Inf).  Scales are power-of-two exponents e stored as UE8M0 bytes e + 127
+// (DeepSeek FP8 §8; FP8-Flow-MoE review, 关键观察 2).
+#pragma once
+
+#include <cuda.h>  // CUtensorMap (type only; the encoder is fetched at run time)
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fp8q.h"
+
+namespace fp8q {
+
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // bounded mbarrier waits: 1 s
+
+// First error wins; later ones are dropped so the reported code is the root cause.
+__device__ __forceinline__ void record_status(int* status, int code) { atomicCAS(status, 0, code); }
+
+// ------------------------------------------------------------------ conversions
+// Two fp32 -> two E4M3 codes, round to nearest even, saturating to +-448; `lo` lands
+// in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two E4M3 codes (low byte first) -> f16x2, exact.
+__device__ __forceinline__ uint32_t cvt_f16x2_e4m3x2(uint32_t two_codes) {
+  uint32_t r;
+  uint16_t v = (uint16_t)two_codes;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+// f16x2 -> two E4M3 codes, round to nearest even, saturating.
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// ------------------------------------------------------------------ scale rule
+// e = the smallest integer with amax <= 448 * 2^e (S = 2^ceil(log2(amax/448))), e = 0
+// for amax == 0, clamped below at -127.  Exact: with amax = mu * 2^p, mu in [1, 2),
+// 448 = 1.75 * 2^8 gives e = p - 8 when mu <= 1.75 and p - 7 otherwise.
+// `amax` is a finite, non-negative fp32.
+__device__ __forceinline__ int tile_exponent(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  if (b == 0u) return 0;
+  const int E = (int)(b >> 23);
+  uint32_t mant = b & 0x7FFFFFu;
+  int p;
+  if (E == 0) {  // fp32 subnormal: renormalize
+    const int L = 31 - __clz((int)mant);
+    p = L - 149;
+    mant = (mant << (23 - L)) & 0x7FFFFFu;
+  } else {
+    p = E - 127;
+  }
+  const int e = p - 8 + (mant > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : e;
+}
+// 2^-e as fp32 for e in [-127, 120] (the exponents this library produces): the
+// exponent field 127 - e lies in [7, 254], so the value is always a normal number.
+__device__ __forceinline__ float exp2_neg(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
+
+// ------------------------------------------------------------------ scaling-aware shift
+// Shift four E4M3 codes of one row by k >= 0 binades: q' = RNE_e4m3(decode(q) * 2^-k)
+// (FP8-Flow-MoE review, 核心方法).
+//  * Fast path (all four exponent fields > k, or k == 0): the result stays normal and
+//    exact, so it is a per-byte subtract of 8k from the exponent field.  The test
+//    (b | 0x80) - 8(k+1) keeps bit 7 set iff the byte's 7-bit magnitude >= 8(k+1),
+//    with no borrow between bytes.
+//  * Otherwise: decode exactly to f16 (every E4M3 value is an f16 value), multiply by
+//    2^-k in f16 and re-encode with round-to-nearest-even.  The f16 product is exact
+//    unless it falls below 2^-20, and every such value rounds to +-0 in E4M3 either
+//    way (the smallest E4M3 rounding threshold is 2^-10), so the result equals the
+//    exact RNE of decode(q) * 2^-k.  For k > 24 the scale is 0 (result +-0).
+__device__ __forceinline__ bool shift_fast_ok(const uint32_t (&w)[4], int k) {
+  const uint32_t thr = (k == 0) ? 0u : (uint32_t)min(k + 1, 16) * 0x08080808u;
+  uint32_t acc = 0x80808080u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc &= (w[i] | 0x80808080u) - thr;
+  return (acc & 0x80808080u) == 0x80808080u;
+}
+__device__ __forceinline__ uint32_t f16_pow2_neg(int k) {  // f16 bits of 2^-k, 0 for k > 24
+  return k <= 14 ? (uint32_t)(15 - k) << 10 : (k <= 24 ? 1u << (24 - k) : 0u);
+}
+__device__ __forceinline__ uint32_t shift_word_general(uint32_t w, uint32_t s2) {
+  const uint32_t lo = mul_f16x2(cvt_f16x2_e4m3x2(w & 0xFFFFu), s2);
+  const uint32_t hi = mul_f16x2(cvt_f16x2_e4m3x2(w >> 16), s2);
+  return cvt_e4m3x2_f16x2(lo) | (cvt_e4m3x2_f16x2(hi) << 16);
+}
+__device__ __forceinline__ void shift_row16(uint32_t (&w)[4], int k) {
+  if (shift_fast_ok(w, k)) {
+    const uint32_t kk = (uint32_t)k * 0x08080808u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] -= kk;
+  } else {
+    const uint32_t s = f16_pow2_neg(k);
+    const uint32_t s2 = s | (s << 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = shift_word_general(w[i], s2);
+  }
+}
+
+// 4x4 byte transpose: out[c] = (r0.byte c, r1.byte c, r2.byte c, r3.byte c).
+__device__ __forceinline__ void transpose4x4(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3, uint32_t& o0,
+                                             uint32_t& o1, uint32_t& o2, uint32_t& o3) {
+  const uint32_t a = __byte_perm(r0, r1, 0x5140), b = __byte_perm(r2, r3, 0x5140);
+  const uint32_t c = __byte_perm(r0, r1, 0x7362), d = __byte_perm(r2, r3, 0x7362);
+  o0 = __byte_perm(a, b, 0x5410);
+  o1 = __byte_perm(a, b, 0x7632);
+  o2 = __byte_perm(c, d, 0x5410);
+  o3 = __byte_perm(c, d, 0x7632);
+}
+
+// ------------------------------------------------------------------ mbarrier / TMA
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase with the given parity to complete; gives up after timeout_ns, or
+// after 2^26 polls should the global timer ever stall.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0; it < (1u << 26); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+  return false;
+}
+// 2-D tiled TMA load (no multicast) of box (x, y) into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------------------ groups
+// Expert groups are contiguous row ranges (DeepSeek FP8 §5.6, M-grouped contiguous):
+// off[0..G], group g = rows off[g]..off[g+1].  Finds the group holding row r and
+// checks everything an address computation relies on: off[g] <= r < off[g+1] <= limit,
+// both ends multiples of 128.  Inconsistent offsets make it return false (the caller
+// records FP8Q_ERR_SHAPE and skips the block), never an out-of-range group.
+__device__ __forceinline__ bool find_group(const int32_t* off, int G, int64_t r, int64_t limit, int64_t& o,
+                                           int64_t& M) {
+  int lo = 0, hi = G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)off[mid] <= r) lo = mid; else hi = mid;
+  }
+  const int64_t a = off[lo], b = off[lo + 1];
+  o = a;
+  M = b - a;
+  return a <= r && r < b && b <= limit && (a & 127) == 0 && (b & 127) == 0;
+}
+// Full consistency check of the offset vector by one CTA (threads stride over the
+// groups): non-decreasing, every group a multiple of 128.  Records FP8Q_ERR_SHAPE.
+// Address safety does not depend on it (find_group bounds every block); it makes
+// inconsistent offsets visible in the status word.
+__device__ __forceinline__ void validate_groups_cta(const int32_t* off, int G, int* status) {
+  bool bad = false;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int64_t a = off[g], b = off[g + 1];
+    bad |= b < a || ((b - a) & 127) != 0;
+  }
+  if (bad) record_status(status, FP8Q_ERR_SHAPE);
+}
+// Rows covered by the groups: off[G] when it is a valid end (multiple of 128 within
+// [0, capacity]), else 0 with FP8Q_ERR_SHAPE recorded.
+__device__ __forceinline__ int64_t grouped_rows(const int32_t* off, int G, int64_t capacity, int* status) {
+  const int64_t first = off[0], last = off[G];
+  if (first != 0 || last < 0 || last > capacity || (last & 127)) {
+    if (status != nullptr) record_status(status, FP8Q_ERR_SHAPE);
+    return 0;
+  }
+  return last;
+}
+
+// ------------------------------------------------------------------ memory
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
+
+}  // namespace fp8q

@@ -1,0 +1,196 @@
+// fp8q_abi.cu — extern "C" entry points of libfp8q: argument checks, per-device facts,
+// the device status word, and dispatch to the kernel launchers.  Every host-detectable
+// error returns before any CUDA call that could touch an output.
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+// The library's only device state: the first device-side error since the last read.
+__device__ int g_fp8q_status = 0;
+
+namespace fp8q {
+
+fp8q_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& d = cache[dev];
+  if (d.device != dev) {
+    DeviceInfo n;
+    n.device = dev;
+    void* p = nullptr;
+    if (cudaDeviceGetAttribute(&n.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaGetSymbolAddress(&p, g_fp8q_status) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    n.status = static_cast<int*>(p);
+    d = n;
+  }
+  *out = d;
+  return FP8Q_OK;
+}
+
+// ---- bounded-wait test hook: one mbarrier nobody arrives at
+__global__ void expire_wait_kernel(uint64_t timeout_ns, int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_bounded(&bar, 0u, timeout_ns)) record_status(status, FP8Q_ERR_TIMEOUT);
+  }
+}
+
+fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream) {
+  expire_wait_kernel<<<1, 32, 0, stream>>>(timeout_ns, dev.status);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+}  // namespace fp8q
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(fp8q_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+constexpr int64_t kMaxDim = 0x7FFFFFFFll;  // TMA coordinates and group offsets are int32
+
+// Shape rules shared by the two transposes.
+fp8q_status check_transpose_args(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols,
+                                 const int32_t* offsets, int32_t num_groups, const uint8_t* qt, const uint8_t* sft) {
+  if (rows < 0 || cols < 0 || cols % 128 || rows > kMaxDim || cols > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (num_groups < 1 || (offsets == nullptr && num_groups != 1)) return FP8Q_ERR_ARG;
+  if (offsets == nullptr && rows % 128) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  if (!q || !sf || !qt || !sft) return FP8Q_ERR_NULL;
+  if (!aligned16(q) || !aligned16(qt) || (offsets && (reinterpret_cast<uintptr_t>(offsets) & 3u))) return FP8Q_ERR_ALIGN;
+  return FP8Q_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fp8q_status_string(fp8q_status s) {
+  switch (s) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_NULL: return "a required pointer is NULL";
+    case FP8Q_ERR_SHAPE: return "sizes violate the layout rules";
+    case FP8Q_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case FP8Q_ERR_ARG: return "invalid argument";
+    case FP8Q_ERR_CUDA: return "a CUDA call failed";
+    case FP8Q_ERR_TIMEOUT: return "a bounded device wait expired";
+    case FP8Q_ERR_DEVICE: return "a kernel saw invalid data";
+  }
+  return "unknown status";
+}
+
+int fp8q_version(void) { return 10000; }
+
+fp8q_status fp8q_last_device_status(fp8q_stream_t stream) {
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return FP8Q_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, dev.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (v != 0 && cudaMemset(dev.status, 0, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return static_cast<fp8q_status>(v);
+}
+
+fp8q_status fp8q_quantize_rowwise(const void* x, int64_t rows, int64_t cols, uint8_t* q, uint8_t* sf,
+                                  fp8q_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 128) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  if (!x || !q || !sf) return FP8Q_ERR_NULL;
+  if (!aligned16(x) || !aligned16(q)) return FP8Q_ERR_ALIGN;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_quantize_tiles(x, rows * (cols / 128), q, sf, as_stream(stream)) == cudaSuccess ? FP8Q_OK
+                                                                                                      : FP8Q_ERR_CUDA;
+}
+
+fp8q_status fp8q_direct_transpose(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols,
+                                  const int32_t* group_offsets, int32_t num_groups, uint8_t* qt, uint8_t* sft,
+                                  fp8q_stream_t stream) {
+  const fp8q_status c = check_transpose_args(q, sf, rows, cols, group_offsets, num_groups, qt, sft);
+  if (c != FP8Q_OK || rows == 0 || cols == 0) return c;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_direct_transpose(dev, q, sf, rows, cols, group_offsets, num_groups, qt, sft, as_stream(stream));
+}
+
+size_t fp8q_naive_workspace_bytes(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return (size_t)(4 * rows * cols);
+}
+
+fp8q_status fp8q_naive_transpose(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols,
+                                 const int32_t* group_offsets, int32_t num_groups, uint8_t* qt, uint8_t* sft,
+                                 void* workspace, size_t workspace_bytes, fp8q_stream_t stream) {
+  const fp8q_status c = check_transpose_args(q, sf, rows, cols, group_offsets, num_groups, qt, sft);
+  if (c != FP8Q_OK || rows == 0 || cols == 0) return c;
+  if (!workspace) return FP8Q_ERR_NULL;
+  if (!aligned16(workspace)) return FP8Q_ERR_ALIGN;
+  if (workspace_bytes < fp8q_naive_workspace_bytes(rows, cols)) return FP8Q_ERR_ARG;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_naive_transpose(dev, q, sf, rows, cols, group_offsets, num_groups, qt, sft, workspace,
+                                      as_stream(stream));
+}
+
+fp8q_status fp8q_swiglu_quant(const void* gate, const void* up, int64_t rows, int64_t cols, uint8_t* q, uint8_t* sf,
+                              uint8_t* qt, uint8_t* sft, fp8q_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 128 || rows > kMaxDim || cols > kMaxDim) return FP8Q_ERR_SHAPE;
+  if ((qt == nullptr) != (sft == nullptr)) return FP8Q_ERR_ARG;
+  if (qt && rows % 128) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  if (!gate || !up || !q || !sf) return FP8Q_ERR_NULL;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(q) || (qt && (reinterpret_cast<uintptr_t>(qt) & 3u)))
+    return FP8Q_ERR_ALIGN;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_swiglu_quant(dev, gate, up, rows, cols, q, sf, qt, sft, as_stream(stream));
+}
+
+size_t fp8q_permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts) {
+  if (tokens < 0 || topk < 1 || num_experts < 1) return 0;
+  return fp8q::permute_workspace_bytes(tokens, topk, num_experts);
+}
+
+fp8q_status fp8q_permute_pad_quant(const void* x, int64_t tokens, int64_t hidden, const int32_t* topk_idx,
+                                   int32_t topk, int32_t num_experts, int32_t align, uint8_t* q, uint8_t* sf,
+                                   int64_t max_out_rows, int32_t* expert_offsets, int32_t* row_id_map,
+                                   void* workspace, size_t workspace_bytes, fp8q_stream_t stream) {
+  if (tokens < 0 || hidden < 0 || hidden % 128 || hidden > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (topk < 1 || topk > 64 || num_experts < 1 || num_experts > 4096 || align < 1 || align > 4096) return FP8Q_ERR_ARG;
+  const int64_t need = tokens * topk + (int64_t)num_experts * (align - 1);
+  if (max_out_rows < need || max_out_rows > kMaxDim) return FP8Q_ERR_ARG;
+  if (!expert_offsets) return FP8Q_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(expert_offsets) & 3u)) return FP8Q_ERR_ALIGN;
+  if (tokens > 0) {
+    if (!topk_idx || !row_id_map || !workspace) return FP8Q_ERR_NULL;
+    if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(topk_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(row_id_map) & 3u))
+      return FP8Q_ERR_ALIGN;
+    if (workspace_bytes < fp8q_permute_workspace_bytes(tokens, topk, num_experts)) return FP8Q_ERR_ARG;
+    if (hidden > 0) {
+      if (!x || !q || !sf) return FP8Q_ERR_NULL;
+      if (!aligned16(x) || !aligned16(q)) return FP8Q_ERR_ALIGN;
+    }
+  }
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_permute_pad_quant(dev, x, tokens, hidden, topk_idx, topk, num_experts, align, q, sf, max_out_rows,
+                                        expert_offsets, row_id_map, workspace, as_stream(stream));
+}
+
+fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream) {
+  if (timeout_ns < 1000ull) timeout_ns = 1000ull;
+  if (timeout_ns > 2000000000ull) timeout_ns = 2000000000ull;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_debug_expire_wait(dev, timeout_ns, as_stream(stream));
+}
+
+}  // extern "C"

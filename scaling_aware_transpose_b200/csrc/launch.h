@@ -1,0 +1,47 @@
+// launch.h — internal (host-side) launchers shared between the C-ABI entry points.
+// Not part of the public ABI; arguments are assumed validated by the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fp8q.h"
+
+namespace fp8q {
+
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int max_smem_optin = 0;
+  int* status = nullptr;  // device address of the status word
+};
+// Per-device facts, queried once per device and cached; also resolves the status
+// word's device address with the device current.
+fp8q_status device_info(DeviceInfo* out);
+
+// Row-wise quantization of n_tiles consecutive 128-element bf16 tiles:
+// x[n_tiles*128] -> q[n_tiles*128], sf[n_tiles].  With limit_rows (a device int32),
+// only the first limit_rows[0] * tiles_per_row tiles are processed.
+cudaError_t launch_quantize_tiles(const void* x, int64_t n_tiles, uint8_t* q, uint8_t* sf, cudaStream_t stream,
+                                  const int32_t* limit_rows = nullptr, int64_t tiles_per_row = 0);
+
+fp8q_status launch_direct_transpose(const DeviceInfo& dev, const uint8_t* q, const uint8_t* sf, int64_t rows,
+                                    int64_t cols, const int32_t* offsets, int32_t num_groups, uint8_t* qt,
+                                    uint8_t* sft, cudaStream_t stream);
+
+fp8q_status launch_naive_transpose(const DeviceInfo& dev, const uint8_t* q, const uint8_t* sf, int64_t rows,
+                                   int64_t cols, const int32_t* offsets, int32_t num_groups, uint8_t* qt,
+                                   uint8_t* sft, void* workspace, cudaStream_t stream);
+
+fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const void* up, int64_t rows, int64_t cols,
+                                uint8_t* q, uint8_t* sf, uint8_t* qt, uint8_t* sft, cudaStream_t stream);
+
+size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts);
+fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,
+                                     const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
+                                     uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,
+                                     int32_t* row_id_map, void* workspace, cudaStream_t stream);
+
+fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace fp8q

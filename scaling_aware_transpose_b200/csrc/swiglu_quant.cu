@@ -1,0 +1,178 @@
+// swiglu_quant.cu — fused SwiGLU + row-wise FP8 quantization (+ direct transpose).
+//
+// FP8-Flow-MoE review, 核心方法 (Fused SwiGLU+Quantization): the activation output is
+// produced directly in FP8 at the activation boundary instead of a BF16 tensor followed
+// by a separate quantize.  Here each CTA owns one 128x128 block: it reads gate and up
+// (bf16) once, computes y = silu(gate) * up in fp32, quantizes each 1x128 row tile with
+// a power-of-two scale, writes the row-wise codes and scales, and, when asked, converts
+// the block to the column-wise layout with the scaling-aware shift before any byte
+// leaves the SM.
+//
+// Arithmetic spec of y (every step one IEEE fp32 operation, round to nearest even, no
+// contraction; identical on every implementation of this spec):
+//   exp(a):  a > 89 -> +inf, a < -104 -> +0; otherwise (Cody & Waite, "Software Manual
+//            for the Elementary Functions", 1980) n = rint(a * L2E),
+//            r = fma(-n, LN2_HI, a), r = fma(-n, LN2_LO, r), p = Horner over 1/k!, k=7..0,
+//            result = (p * 2^floor(n/2)) * 2^(n - floor(n/2));
+//   silu(g) = g / (1 + exp(-g));   y = silu(g) * u.
+// Constants (each derived from its definition): L2E = fp32(log2 e); LN2_HI = ln 2 cut
+// to the top 15 mantissa bits; LN2_LO = fp32(ln 2 - LN2_HI); 1/k! rounded to fp32.
+#include "common.cuh"
+#include "launch.h"
+
+namespace fp8q {
+namespace {
+
+constexpr float kL2E = 0x1.715476p+0f;
+constexpr float kLn2Hi = 0x1.62e4p-1f;
+constexpr float kLn2Lo = 0x1.7f7d1cp-20f;
+constexpr float kC0 = 0x1p+0f, kC1 = 0x1p+0f, kC2 = 0x1p-1f, kC3 = 0x1.555556p-3f;  // 1/k!
+constexpr float kC4 = 0x1.555556p-5f, kC5 = 0x1.111112p-7f, kC6 = 0x1.6c16c2p-10f, kC7 = 0x1.a01a02p-13f;
+
+__device__ __forceinline__ float exp_spec(float a) {
+  const float ac = fminf(fmaxf(a, -104.0f), 89.0f);  // keeps n in [-150, 128]
+  const float n = rintf(__fmul_rn(ac, kL2E));
+  float r = __fmaf_rn(-n, kLn2Hi, ac);
+  r = __fmaf_rn(-n, kLn2Lo, r);
+  float p = kC7;
+  p = __fmaf_rn(p, r, kC6);
+  p = __fmaf_rn(p, r, kC5);
+  p = __fmaf_rn(p, r, kC4);
+  p = __fmaf_rn(p, r, kC3);
+  p = __fmaf_rn(p, r, kC2);
+  p = __fmaf_rn(p, r, kC1);
+  p = __fmaf_rn(p, r, kC0);
+  const int ni = (int)n;
+  const int n1 = ni >> 1;  // floor(n / 2)
+  const int n2 = ni - n1;
+  const float res = __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
+  return a > 89.0f ? __int_as_float(0x7F800000) : (a < -104.0f ? 0.0f : res);
+}
+
+__device__ __forceinline__ float swiglu_spec(float g, float u) {
+  const float den = __fadd_rn(1.0f, exp_spec(-g));
+  return __fmul_rn(__fdiv_rn(g, den), u);
+}
+
+constexpr int kThreads = 256;
+constexpr int kPasses = 4;  // 4 passes x 32 rows x (8 threads x 16 elements)
+
+__device__ __forceinline__ uint32_t swizzled_chunk(int row, int chunk) { return (uint32_t)(chunk ^ ((row >> 2) & 7)); }
+
+__global__ void __launch_bounds__(kThreads) swiglu_quant_kernel(const uint16_t* __restrict__ gate,
+                                                                const uint16_t* __restrict__ up, int64_t rows, int cols,
+                                                                uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                                                                uint8_t* __restrict__ qt, uint8_t* __restrict__ sft) {
+  __shared__ __align__(16) uint8_t tile[128 * 128];
+  __shared__ __align__(16) uint8_t e_row[128];
+  __shared__ int e_max_sh;
+  const int tid = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.x * 128;  // row block (grid.x has the larger range)
+  const int c0 = blockIdx.y * 128;
+  const int ncb = cols >> 7;
+  const int sub = tid & 7;      // 16-element chunk of the row tile
+  const int rsub = tid >> 3;    // row within a pass (0..31)
+
+  // ---- load gate/up for all passes first (memory-level parallelism)
+  uint4 gv[kPasses][2], uv[kPasses][2];
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) {
+    const int64_t r = r0 + p * 32 + rsub;
+    if (r < rows) {
+      const int64_t base = r * cols + c0 + sub * 16;
+      gv[p][0] = ld_stream(reinterpret_cast<const uint4*>(gate + base));
+      gv[p][1] = ld_stream(reinterpret_cast<const uint4*>(gate + base + 8));
+      uv[p][0] = ld_stream(reinterpret_cast<const uint4*>(up + base));
+      uv[p][1] = ld_stream(reinterpret_cast<const uint4*>(up + base + 8));
+    } else {
+      gv[p][0] = gv[p][1] = uv[p][0] = uv[p][1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  // ---- y, row-wise quantization
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) {
+    const int rl = p * 32 + rsub;
+    const int64_t r = r0 + rl;
+    float y[16];
+    const uint32_t gw[8] = {gv[p][0].x, gv[p][0].y, gv[p][0].z, gv[p][0].w, gv[p][1].x, gv[p][1].y, gv[p][1].z, gv[p][1].w};
+    const uint32_t uw[8] = {uv[p][0].x, uv[p][0].y, uv[p][0].z, uv[p][0].w, uv[p][1].x, uv[p][1].y, uv[p][1].z, uv[p][1].w};
+    uint32_t amax = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      y[2 * k] = swiglu_spec(__uint_as_float(gw[k] << 16), __uint_as_float(uw[k] << 16));
+      y[2 * k + 1] = swiglu_spec(__uint_as_float(gw[k] & 0xFFFF0000u), __uint_as_float(uw[k] & 0xFFFF0000u));
+      amax = max(amax, max(__float_as_uint(y[2 * k]) & 0x7FFFFFFFu, __float_as_uint(y[2 * k + 1]) & 0x7FFFFFFFu));
+    }
+#pragma unroll
+    for (int o = 4; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    const int e = tile_exponent(__uint_as_float(amax));
+    const float s = exp2_neg(e);
+    uint4 codes;
+    codes.x = cvt_e4m3x2_f32(y[0] * s, y[1] * s) | (cvt_e4m3x2_f32(y[2] * s, y[3] * s) << 16);
+    codes.y = cvt_e4m3x2_f32(y[4] * s, y[5] * s) | (cvt_e4m3x2_f32(y[6] * s, y[7] * s) << 16);
+    codes.z = cvt_e4m3x2_f32(y[8] * s, y[9] * s) | (cvt_e4m3x2_f32(y[10] * s, y[11] * s) << 16);
+    codes.w = cvt_e4m3x2_f32(y[12] * s, y[13] * s) | (cvt_e4m3x2_f32(y[14] * s, y[15] * s) << 16);
+    if (r < rows) {
+      *reinterpret_cast<uint4*>(q + r * cols + c0 + sub * 16) = codes;
+      if (sub == 0) sf[r * ncb + (c0 >> 7)] = (uint8_t)(e + 127);
+    }
+    if (qt != nullptr) {
+      *reinterpret_cast<uint4*>(tile + rl * 128 + (swizzled_chunk(rl, sub) << 4)) = codes;
+      if (sub == 0) e_row[rl] = (uint8_t)(e + 127);
+    }
+  }
+  if (qt == nullptr) return;  // uniform across the CTA
+
+  // ---- direct transpose of the block (rows % 128 == 0 is guaranteed by the host)
+  __syncthreads();
+  if (tid < 32) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(e_row)[tid];
+    int m = (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (tid == 0) e_max_sh = m;
+  }
+  __syncthreads();
+  const int emax = e_max_sh;
+  const int lane = tid & 31, c = tid >> 5;  // token quad = lane, 16-byte column chunk = warp
+  const uint32_t ew = reinterpret_cast<const uint32_t*>(e_row)[lane];
+  uint32_t w[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rl = 4 * lane + i;
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + rl * 128 + (swizzled_chunk(rl, c) << 4));
+    w[i][0] = v.x;
+    w[i][1] = v.y;
+    w[i][2] = v.z;
+    w[i][3] = v.w;
+    shift_row16(w[i], emax - (int)((ew >> (8 * i)) & 0xFFu));
+  }
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    uint32_t o0, o1, o2, o3;
+    transpose4x4(w[0][qq], w[1][qq], w[2][qq], w[3][qq], o0, o1, o2, o3);
+    const int64_t ch = c0 + 16 * c + 4 * qq;
+    uint8_t* dst = qt + ch * rows + r0 + 4 * lane;
+    *reinterpret_cast<uint32_t*>(dst) = o0;
+    *reinterpret_cast<uint32_t*>(dst + rows) = o1;
+    *reinterpret_cast<uint32_t*>(dst + 2 * rows) = o2;
+    *reinterpret_cast<uint32_t*>(dst + 3 * rows) = o3;
+  }
+  if (tid < 128) sft[(int64_t)(c0 + tid) * (rows >> 7) + (r0 >> 7)] = (uint8_t)emax;
+}
+
+}  // namespace
+
+fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const void* up, int64_t rows, int64_t cols,
+                                uint8_t* q, uint8_t* sf, uint8_t* qt, uint8_t* sft, cudaStream_t stream) {
+  (void)dev;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  const int64_t gx = (rows + 127) / 128;
+  if (gx > 0x7FFFFFFF || cols / 128 > 65535) return FP8Q_ERR_SHAPE;
+  dim3 grid((unsigned)gx, (unsigned)(cols / 128));
+  swiglu_quant_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(gate),
+                                                     static_cast<const uint16_t*>(up), rows, (int)cols, q, sf, qt, sft);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+}  // namespace fp8q

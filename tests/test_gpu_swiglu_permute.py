@@ -1,0 +1,134 @@
+"""GPU parity: fused SwiGLU+quantize (+ direct transpose), fused permute+pad+quantize and
+the grouped direct transpose on its output, against the CPU oracle, byte for byte."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scaling_aware_transpose_b200 as sat
+from scaling_aware_transpose_b200 import synthetic
+from gpu_helpers import assert_bytes_equal, dev, device_status_ok, host
+
+pytestmark = pytest.mark.gpu
+
+
+def check_swiglu(d, transposed=True):
+    q, sf, qt, sft = sat.swiglu_quant(dev(d["gate"]), dev(d["up"]), transposed=transposed)
+    device_status_ok()
+    oq, osf, oqt, osft = oracle.swiglu_quant(d["gate"], d["up"], transposed=transposed)
+    assert_bytes_equal(host(sf), osf, "SF")
+    assert_bytes_equal(host(q), oq, "Q")
+    if transposed:
+        assert_bytes_equal(host(sft), osft, "SF^T")
+        assert_bytes_equal(host(qt), oqt, "Q^T")
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (640, 1024), (1024, 2048)])
+def test_swiglu_shapes(rows, cols):
+    check_swiglu(synthetic.swiglu(rows=rows, cols=cols, seed=rows + 3 * cols))
+
+
+def test_swiglu_rowwise_only_ragged_rows():
+    check_swiglu(synthetic.swiglu(rows=300, cols=256, seed=5), transposed=False)
+
+
+def test_swiglu_exp_range_edges():
+    """Gate values that reach the exp spec's clamps and the division's extremes."""
+    rows, cols = 128, 256
+    g = np.linspace(-120, 120, rows * cols, dtype=np.float32).reshape(rows, cols)
+    u = np.ones((rows, cols), np.float32)
+    u[::2] = -3.0
+    d = {"gate": synthetic._bf16_bits(g), "up": synthetic._bf16_bits(u)}
+    check_swiglu(d)
+
+
+def test_swiglu_config_full():
+    check_swiglu(synthetic.swiglu())
+
+
+# ------------------------------------------------------------------ permute
+
+def check_permute(d, E, align):
+    x, idx = d["x"], d["topk_idx"]
+    q, sf, off, rmap = sat.permute_pad_quant(dev(x), dev(idx), E, align)
+    device_status_ok()
+    oq, osf, ooff, ormap = oracle.permute_pad_quant(x, idx, E, align)
+    assert_bytes_equal(host(off), ooff, "expert offsets")
+    assert_bytes_equal(host(rmap), ormap, "row_id_map")
+    n = int(ooff[-1])
+    assert_bytes_equal(host(sf)[:n], osf[:n], "SF")
+    assert_bytes_equal(host(q)[:n], oq[:n], "Q")
+    return q, sf, off, oq, osf, ooff
+
+
+@pytest.mark.parametrize("tokens,hidden,E,K,align", [(8, 128, 4, 2, 16), (100, 256, 8, 2, 16),
+                                                      (512, 384, 32, 8, 128), (3000, 256, 16, 4, 1),
+                                                      (1500, 512, 7, 3, 64)])
+def test_permute_shapes(tokens, hidden, E, K, align):
+    rng = np.random.default_rng(tokens)
+    d = {"x": synthetic.scaled_normal(tokens, hidden, seed=tokens + 1),
+         "topk_idx": synthetic.zipf_topk(tokens, E, K, rng)}
+    check_permute(d, E, align)
+
+
+def test_permute_with_duplicate_and_skewed_routing():
+    tokens, hidden, E = 700, 256, 5
+    idx = np.zeros((tokens, 3), np.int32)
+    idx[:, 1] = 0           # every token sends two slots to expert 0
+    idx[::7, 2] = 4
+    d = {"x": synthetic.scaled_normal(tokens, hidden, seed=9), "topk_idx": idx}
+    check_permute(d, E, 128)
+
+
+def test_permute_bad_index_sets_device_status():
+    x = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")
+    idx = torch.tensor([[0], [1], [9], [2]], dtype=torch.int32, device="cuda")
+    sat.permute_pad_quant(x, idx, 4, 16)
+    assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE
+
+
+def test_permute_zero_tokens():
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((0, 8), dtype=torch.int32, device="cuda")
+    q, sf, off, rmap = sat.permute_pad_quant(x, idx, 32, 128)
+    device_status_ok()
+    assert torch.all(off == 0)
+
+
+def test_moe_config_permute_then_grouped_transpose():
+    """The MoE workload end to end: permute+pad(128)+quantize, then the grouped direct
+    transpose on the device-resident offsets; transposed output checked on every group's
+    first and last block and on a seeded sample of the rest."""
+    d = synthetic.moe()
+    q, sf, off, oq, osf, ooff = check_permute(d, 32, 128)
+    qt, sft = sat.direct_transpose(q, sf, off)
+    device_status_ok()
+    H = q.shape[1]
+    qt_h, sft_h = host(qt), host(sft)
+    rng = np.random.default_rng(0)
+    blocks = set()
+    for g in range(32):
+        a, b = int(ooff[g]), int(ooff[g + 1])
+        if a == b:
+            continue
+        blocks |= {a // 128, b // 128 - 1}
+        blocks |= set(rng.integers(a // 128, b // 128, size=4).tolist())
+    for blk in sorted(blocks):
+        g = int(np.searchsorted(ooff, blk * 128, side="right") - 1)
+        a, b = int(ooff[g]), int(ooff[g + 1])
+        M = b - a
+        r0 = blk * 128
+        want_qt, want_sft = oracle.direct_transpose(oq[r0:r0 + 128], osf[r0:r0 + 128])
+        got = qt_h[H * a: H * a + H * M].reshape(H, M)[:, r0 - a: r0 - a + 128]
+        assert_bytes_equal(got, want_qt, f"grouped Q^T block {blk}")
+        gs = sft_h[H * a // 128: H * a // 128 + H * M // 128].reshape(H, M // 128)[:, (r0 - a) // 128]
+        assert_bytes_equal(gs, want_sft[:, 0], f"grouped SF^T block {blk}")
+
+
+def test_bounded_wait_expires_cleanly():
+    sat.fp8q_debug_expire_wait(2_000_000)  # 2 ms, nobody arrives
+    assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_TIMEOUT
+    # the context is still usable
+    x = dev(synthetic.scaled_normal(128, 128, seed=1))
+    q, sf = sat.quantize_rowwise(x)
+    device_status_ok()
