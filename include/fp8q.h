@@ -153,6 +153,34 @@ fp8q_status fp8q_permute_pad_quant(const void *x, int64_t tokens, int64_t hidden
                                    int32_t *row_id_map, void *workspace, size_t workspace_bytes,
                                    fp8q_stream_t stream);
 
+/* Size of the library's static scratch for fp8q_permute_pad_quant_noalloc (4 MiB). */
+#define FP8Q_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* fp8q_permute_pad_quant for callers that cannot allocate device memory (the paper has
+ * no counterpart: this is a deployment convenience).  Some callers cannot call
+ * cudaMalloc where they route tokens: their device memory belongs to an allocator they
+ * cannot reach from this point, or they run under a fixed, pre-planned memory budget, or
+ * they are a plugin handed only its input and output buffers.  This entry point takes
+ * the same arguments as fp8q_permute_pad_quant minus the workspace, and keeps the
+ * routing scratch in a file-scope device array of FP8Q_NOALLOC_SCRATCH_BYTES instead.
+ * It allocates nothing and calls no allocating routine.
+ *   Limit: fp8q_permute_workspace_bytes(tokens, topk, num_experts) must not exceed
+ *   FP8Q_NOALLOC_SCRATCH_BYTES (about tokens*topk*num_experts/128 bytes; e.g. 2M
+ *   token-slot pairs with 256 experts, or 16M with 32); larger requests return
+ *   FP8Q_ERR_ARG before any CUDA call.
+ *   Memory: every GPU that loads the library holds the array until the process exits.
+ *   Set-up: the first call on each device resolves the array's device address (with
+ *   that device current); make that first call before capturing a stream.
+ *   Sharing: all calls on a device use the same array, which keeps the previous call's
+ *   contents (nothing in it needs to start at zero: every word is written before it is
+ *   read).  Calls that overlap on the GPU (other streams, other threads) race on it:
+ *   order them on one stream.
+ * Other arguments, results and errors: as fp8q_permute_pad_quant. */
+fp8q_status fp8q_permute_pad_quant_noalloc(const void *x, int64_t tokens, int64_t hidden,
+                                           const int32_t *topk_idx, int32_t topk, int32_t num_experts,
+                                           int32_t align, uint8_t *q, uint8_t *sf, int64_t max_out_rows,
+                                           int32_t *expert_offsets, int32_t *row_id_map, fp8q_stream_t stream);
+
 /* Test hook for the bounded-wait machinery (no counterpart on the pages): launches one
  * CTA that waits on an mbarrier nobody arrives at, giving up after `timeout_ns`
  * nanoseconds (clamped to [1e3, 2e9]); the kernel then records FP8Q_ERR_TIMEOUT in the

@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
             "fp8q_swiglu_quant": ([P, P, I64, I64, P, P, P, P, P], ctypes.c_int),
             "fp8q_permute_workspace_bytes": ([I64, I32, I32], SZ),
             "fp8q_permute_pad_quant": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
+            "fp8q_permute_pad_quant_noalloc": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P], ctypes.c_int),
             "fp8q_debug_expire_wait": ([ctypes.c_uint64, P], ctypes.c_int),
             "fp8q_version": ([], ctypes.c_int),
         }
@@ -142,6 +143,20 @@ def fp8q_permute_pad_quant(x, tokens: int, hidden: int, topk_idx, topk: int, num
                                         _ptr(q), _ptr(sf), max_out_rows, _ptr(expert_offsets),
                                         _ptr(row_id_map), _ptr(workspace), workspace_bytes,
                                         _stream(stream)), "fp8q_permute_pad_quant")
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20  # FP8Q_NOALLOC_SCRATCH_BYTES
+
+
+def fp8q_permute_pad_quant_noalloc(x, tokens: int, hidden: int, topk_idx, topk: int, num_experts: int,
+                                   align: int, q, sf, max_out_rows: int, expert_offsets, row_id_map,
+                                   stream=None) -> None:
+    """fp8q_permute_pad_quant without a workspace argument: the routing scratch lives in the
+    library's static device array (for callers that cannot allocate device memory)."""
+    _check(lib().fp8q_permute_pad_quant_noalloc(_ptr(x), tokens, hidden, _ptr(topk_idx), topk, num_experts,
+                                                align, _ptr(q), _ptr(sf), max_out_rows, _ptr(expert_offsets),
+                                                _ptr(row_id_map), _stream(stream)),
+           "fp8q_permute_pad_quant_noalloc")
 
 
 def fp8q_debug_expire_wait(timeout_ns: int, stream=None) -> None:
