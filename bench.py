@@ -165,6 +165,104 @@ def cpu_baseline(x_bits, budget_s: float = 10.0, max_reps: int = 50):
                                         f"{reps} repetitions, {sum(times):.1f} s"}
 
 
+
+def time_on_stream(fn, reps, stream, before=None):
+    """Median device time (s) of fn() over reps launches, each bracketed by CUDA events on
+    `stream`; `before` (e.g. an L2 flush) runs outside the events."""
+    import torch
+    pairs = []
+    for _ in range(reps):
+        if before is not None:
+            before()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        pairs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) * 1e-3 for a, b in pairs)
+
+
+def measure_workloads(reps, device, stream, flush, peak):
+    """The other hot-path rows on their own workloads, each kernel after an L2 flush:
+    fused SwiGLU+quantize(+transpose) on gate/up [32768, 2048]; fused permute+pad(128)+
+    quantize of X [16384, 7168] with top-8 of 32 Zipf(1.1) experts, then the grouped
+    direct transpose on its device offsets; quantize + direct transpose on the range-
+    stress X [65536, 7168]."""
+    import torch
+
+    import scaling_aware_transpose_b200 as sat
+    from scaling_aware_transpose_b200 import synthetic
+    sp = stream.cuda_stream
+
+    def entry(nbytes, t):
+        gbs = nbytes / t / 1e9
+        return {"us": round(t * 1e6, 2), "bytes": int(nbytes), "GB/s": round(gbs, 1),
+                "frac_of_peak": round(gbs / peak, 4)}
+
+    out = {}
+    # SwiGLU
+    d = synthetic.swiglu()
+    g = synthetic.to_torch_bf16(d["gate"]).to(device)
+    u = synthetic.to_torch_bf16(d["up"]).to(device)
+    R, C = g.shape
+    n = R * C
+    q = torch.empty((R, C), dtype=torch.uint8, device=device)
+    sf = torch.empty((R, C // 128), dtype=torch.uint8, device=device)
+    qt = torch.empty((C, R), dtype=torch.uint8, device=device)
+    sft = torch.empty((C, R // 128), dtype=torch.uint8, device=device)
+    t = time_on_stream(lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, qt, sft, sp), reps + 2, stream,
+                       lambda: flush.fill_(5))
+    t_row = time_on_stream(lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, None, None, sp), reps + 2, stream,
+                           lambda: flush.fill_(5))
+    out["swiglu_quant [32768x2048] (+transpose)"] = entry(4 * n + 2 * (n + n // 128), t)
+    out["swiglu_quant [32768x2048] (row-wise only)"] = entry(4 * n + n + n // 128, t_row)
+    del g, u, q, sf, qt, sft
+    # MoE: permute + pad + quantize, grouped direct transpose
+    d = synthetic.moe()
+    x = synthetic.to_torch_bf16(d["x"]).to(device)
+    idx = torch.from_numpy(d["topk_idx"]).to(device)
+    T, H = x.shape
+    K, E, align = idx.shape[1], d["num_experts"], 128
+    max_rows = sat.permute_max_rows(T, K, E, align)
+    q = torch.empty((max_rows, H), dtype=torch.uint8, device=device)
+    sf = torch.empty((max_rows, H // 128), dtype=torch.uint8, device=device)
+    off = torch.empty(E + 1, dtype=torch.int32, device=device)
+    rmap = torch.empty(T * K, dtype=torch.int32, device=device)
+    ws = torch.empty(sat.fp8q_permute_workspace_bytes(T, K, E), dtype=torch.uint8, device=device)
+    perm = lambda: sat.fp8q_permute_pad_quant(x, T, H, idx, K, E, align, q, sf, max_rows, off, rmap, ws,
+                                              ws.numel(), sp)
+    t_perm = time_on_stream(perm, reps + 2, stream, lambda: flush.fill_(6))
+    R = int(off[-1].item())
+    qt = torch.empty(max_rows * H, dtype=torch.uint8, device=device)
+    sft = torch.empty(max_rows * H // 128, dtype=torch.uint8, device=device)
+    t_gt = time_on_stream(lambda: sat.fp8q_direct_transpose(q, sf, max_rows, H, off, E, qt, sft, sp), reps + 2,
+                          stream, lambda: flush.fill_(7))
+    perm_bytes = 2 * T * H + 4 * T * K + R * (H + H // 128) + 4 * (E + 1) + 4 * T * K
+    out[f"permute_pad_quant [16384x7168] top8/32 -> {R} rows"] = entry(perm_bytes, t_perm)
+    out[f"direct_transpose grouped [{R}x7168] 32 experts"] = entry(2 * R * (H + H // 128), t_gt)
+    del x, idx, q, sf, off, rmap, ws, qt, sft
+    # range stress
+    d = synthetic.stress()
+    x = synthetic.to_torch_bf16(d["x"]).to(device)
+    R, C = x.shape
+    n = R * C
+    q = torch.empty((R, C), dtype=torch.uint8, device=device)
+    sf = torch.empty((R, C // 128), dtype=torch.uint8, device=device)
+    qt = torch.empty((C, R), dtype=torch.uint8, device=device)
+    sft = torch.empty((C, R // 128), dtype=torch.uint8, device=device)
+    t_q = time_on_stream(lambda: sat.fp8q_quantize_rowwise(x, R, C, q, sf, sp), reps + 2, stream,
+                         lambda: flush.fill_(8))
+    t_d = time_on_stream(lambda: sat.fp8q_direct_transpose(q, sf, R, C, None, 1, qt, sft, sp), reps + 2, stream,
+                         lambda: flush.fill_(9))
+    out["quantize_rowwise stress [65536x7168]"] = entry(3 * n + n // 128, t_q)
+    out["direct_transpose stress [65536x7168]"] = entry(2 * n + 2 * (n // 128), t_d)
+    status = sat.fp8q_last_device_status(sp)
+    if status != 0:
+        raise RuntimeError(f"device status {sat.STATUS.get(status)} in the workload measurements")
+    return out
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, rank, world, local_rank):
     import numpy as np
@@ -261,6 +359,14 @@ def run_ours(args, rank, world, local_rank):
     t_chain = statistics.median(a.elapsed_time(b) * 1e-3 for a, b in chained)
     t_naive = statistics.median(a.elapsed_time(b) * 1e-3 for a, b in naive)
 
+    # same two kernels after a flush that leaves no dirty lines (write, then read the
+    # flush buffer): the kernel does not pay for writing back data it never touched
+    def clean_flush():
+        flush.fill_(5)
+        flush.sum(dtype=torch.int32)
+    t_q_clean = time_on_stream(quant, min(K, 50), stream, clean_flush)
+    t_d_clean = time_on_stream(direct, min(K, 50), stream, clean_flush)
+
     # ---- end to end through the C ABI from pinned host buffers
     q_h = torch.empty_like(q, device="cpu").pin_memory()
     sf_h = torch.empty_like(sf, device="cpu").pin_memory()
@@ -316,6 +422,10 @@ def run_ours(args, rank, world, local_rank):
                                       "direct_speedup": round(t_naive / avg_d, 2)},
             "chained_step_no_flush_between": {"us": round(t_chain * 1e6, 2),
                                               "GB/s": round(BYTES_STEP / t_chain / 1e9, 1)},
+            "clean_l2_flush": {"quantize_us": round(t_q_clean * 1e6, 2),
+                               "quantize_GB/s": round(BYTES_QUANT / t_q_clean / 1e9, 1),
+                               "direct_us": round(t_d_clean * 1e6, 2),
+                               "direct_GB/s": round(BYTES_DIRECT / t_d_clean / 1e9, 1)},
         },
         "gpu_launches": 2 * K,
         "e2e": {"value": round(BYTES_STEP / t_e2e / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": 2 * N_ELEM,
@@ -323,6 +433,8 @@ def run_ours(args, rank, world, local_rank):
                 "result_matches_device": ok_e2e},
         "clocks": clocks.summary(),
     }
+    if not args.no_extras:
+        line["workloads"] = measure_workloads(min(K, 20), device, stream, flush, peak)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x_bits, budget_s=args.cpu_budget)
     return line
@@ -359,6 +471,33 @@ def run_reference(args):
     }
 
 
+# ------------------------------------------------------------------ ncu driver
+def run_profile(args):
+    """Launches only one kernel, --warmup + --steps times back to back on the dense workload
+    (no flush, no timing): the command line that the committed ncu summaries capture."""
+    import torch
+
+    import scaling_aware_transpose_b200 as sat
+    from scaling_aware_transpose_b200 import synthetic
+    torch.cuda.set_device(0)
+    x = synthetic.to_torch_bf16(synthetic.dense(seed=0)["x"]).cuda()
+    q, sf = sat.quantize_rowwise(x)
+    qt, sft = sat.direct_transpose(q, sf)
+    ws = torch.empty(sat.fp8q_naive_workspace_bytes(ROWS, COLS), dtype=torch.uint8, device="cuda")
+    calls = {
+        "quantize": lambda: sat.fp8q_quantize_rowwise(x, ROWS, COLS, q, sf),
+        "direct": lambda: sat.fp8q_direct_transpose(q, sf, ROWS, COLS, None, 1, qt, sft),
+        "naive": lambda: sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, ws, ws.numel()),
+    }
+    torch.cuda.synchronize()
+    for _ in range(args.warmup + args.steps):
+        calls[args.profile]()
+    torch.cuda.synchronize()
+    st = sat.fp8q_last_device_status()
+    print(json.dumps({"profile": args.profile, "launches": args.warmup + args.steps, "status": st}))
+    return 0 if st == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,9 +505,14 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-extras", action="store_true", help="skip the SwiGLU / MoE / stress workload timings")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
+    ap.add_argument("--profile", choices=["quantize", "direct", "naive"], default=None,
+                    help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)
+    if args.profile:
+        return run_profile(args)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

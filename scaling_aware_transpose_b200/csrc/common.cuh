@@ -71,17 +71,18 @@ __device__ __forceinline__ int tile_exponent(float amax) {
 __device__ __forceinline__ float exp2_neg(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
 
 // ------------------------------------------------------------------ scaling-aware shift
-// Shift four E4M3 codes of one row by k >= 0 binades: q' = RNE_e4m3(decode(q) * 2^-k)
+// Shift E4M3 codes of one row by k >= 0 binades: q' = RNE_e4m3(decode(q) * 2^-k)
 // (FP8-Flow-MoE review, 核心方法).
-//  * Fast path (all four exponent fields > k, or k == 0): the result stays normal and
-//    exact, so it is a per-byte subtract of 8k from the exponent field.  The test
-//    (b | 0x80) - 8(k+1) keeps bit 7 set iff the byte's 7-bit magnitude >= 8(k+1),
-//    with no borrow between bytes.
-//  * Otherwise: decode exactly to f16 (every E4M3 value is an f16 value), multiply by
-//    2^-k in f16 and re-encode with round-to-nearest-even.  The f16 product is exact
-//    unless it falls below 2^-20, and every such value rounds to +-0 in E4M3 either
-//    way (the smallest E4M3 rounding threshold is 2^-10), so the result equals the
-//    exact RNE of decode(q) * 2^-k.  For k > 24 the scale is 0 (result +-0).
+//  * General form, used for every word: decode exactly to f16 (every E4M3 value is an
+//    f16 value), multiply by 2^-k in f16 and re-encode with round-to-nearest-even.
+//    While the result stays normal this is the exponent-field subtract; where it turns
+//    subnormal the hardware re-rounds the mantissa.  The f16 product is exact unless it
+//    falls below 2^-20, and every such value rounds to +-0 in E4M3 either way (the
+//    smallest E4M3 rounding threshold is 2^-10), so the result equals the exact RNE of
+//    decode(q) * 2^-k.  For k > 24 the scale is 0 (result +-0, sign kept).
+//  * SWAR form (all four exponent fields > k, or k == 0): a per-byte subtract of 8k.
+//    The test (b | 0x80) - 8(k+1) keeps bit 7 set iff the byte's 7-bit magnitude is
+//    >= 8(k+1), with no borrow between bytes.
 __device__ __forceinline__ bool shift_fast_ok(const uint32_t (&w)[4], int k) {
   const uint32_t thr = (k == 0) ? 0u : (uint32_t)min(k + 1, 16) * 0x08080808u;
   uint32_t acc = 0x80808080u;
@@ -92,19 +93,35 @@ __device__ __forceinline__ bool shift_fast_ok(const uint32_t (&w)[4], int k) {
 __device__ __forceinline__ uint32_t f16_pow2_neg(int k) {  // f16 bits of 2^-k, 0 for k > 24
   return k <= 14 ? (uint32_t)(15 - k) << 10 : (k <= 24 ? 1u << (24 - k) : 0u);
 }
-__device__ __forceinline__ uint32_t shift_word_general(uint32_t w, uint32_t s2) {
-  const uint32_t lo = mul_f16x2(cvt_f16x2_e4m3x2(w & 0xFFFFu), s2);
-  const uint32_t hi = mul_f16x2(cvt_f16x2_e4m3x2(w >> 16), s2);
-  return cvt_e4m3x2_f16x2(lo) | (cvt_e4m3x2_f16x2(hi) << 16);
+__device__ __forceinline__ uint32_t f16x2_pow2_neg(int k) {
+  const uint32_t s = f16_pow2_neg(k);
+  return s | (s << 16);
 }
+// Four codes (one row) times the f16x2 scale s2 = {2^-k, 2^-k}, re-encoded.
+__device__ __forceinline__ uint32_t shift_word_general(uint32_t w, uint32_t s2) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h, ol, oh;\n\t.reg .b32 fl, fh;\n\t"
+      "mov.b32 {l, h}, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 fl, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 fh, h;\n\t"
+      "mul.rn.f16x2 fl, fl, %2;\n\t"
+      "mul.rn.f16x2 fh, fh, %2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 ol, fl;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 oh, fh;\n\t"
+      "mov.b32 %0, {ol, oh};\n\t}"
+      : "=r"(r)
+      : "r"(w), "r"(s2));
+  return r;
+}
+// One 16-byte row chunk: the SWAR subtract when it is exact for every byte, else the
+// general form (per-lane branch; used where rows rarely need re-rounding).
 __device__ __forceinline__ void shift_row16(uint32_t (&w)[4], int k) {
   if (shift_fast_ok(w, k)) {
     const uint32_t kk = (uint32_t)k * 0x08080808u;
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] -= kk;
   } else {
-    const uint32_t s = f16_pow2_neg(k);
-    const uint32_t s2 = s | (s << 16);
+    const uint32_t s2 = f16x2_pow2_neg(k);
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = shift_word_general(w[i], s2);
   }

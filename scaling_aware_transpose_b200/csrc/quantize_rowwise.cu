@@ -6,9 +6,11 @@
 //
 // HBM-bound streaming kernel (3 bytes moved per element plus 1 per 128).  Layout: a
 // row-major [rows, cols] tensor with cols % 128 == 0 is a flat sequence of 128-element
-// tiles, so the kernel runs over tiles: 16 lanes per tile, 8 bf16 (one 16-byte load)
-// per lane, two tiles per warp per slot, UNROLL slots per thread with every load issued
-// before any use.  Loads are coalesced 512-byte warp segments, stores 256-byte ones.
+// tiles, so the kernel runs over tiles: 8 lanes per tile, 16 bf16 (two 16-byte loads)
+// per lane, four tiles per warp per slot, two slots per thread with every load issued
+// before any use.  Instruction budget matters here (the integer ALU pipe is the first
+// to saturate): the amax uses packed bf16x2 max-of-magnitudes, three shuffles, an
+// exponent read straight off the BF16 bits, and packed f32x2 multiplies.
 #include "common.cuh"
 #include "launch.h"
 
@@ -16,26 +18,45 @@ namespace fp8q {
 namespace {
 
 constexpr int kQThreads = 256;
-constexpr int kQUnroll = 4;
+constexpr int kQUnroll = 2;        // tile slots per thread, all loads issued first
+constexpr int kTilesPerWarp = 4;   // 8 lanes per tile, 16 elements per lane
 
-// Max of the 8 bf16 magnitudes in `v`, as the fp32 bit pattern (non-negative floats
-// order like their bit patterns, so an unsigned 16-bit max is a float max).
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4& v) {
-  const uint32_t m0 = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-  const uint32_t m1 = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
-  const uint32_t m = __vmaxu2(m0, m1);
-  return max(m & 0xFFFFu, m >> 16) << 16;
+// Two bf16x2 words -> the larger magnitude per half (sign bits meaningless).
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
+// Scale exponent of a tile from its BF16 amax bit pattern (sign clear): e = the smallest
+// integer with amax <= 448 * 2^e, 0 for amax == 0, clamped below at -127.  With
+// amax = (1 + m/128) * 2^(E-127): e = E - 135, plus one when the 7-bit mantissa exceeds
+// 0x60 (mu > 1.75 = 448 / 2^8).  BF16 subnormals (E == 0) are all far below the clamp.
+__device__ __forceinline__ int bf16_tile_exponent(uint32_t amax16) {
+  const int e = (int)(amax16 >> 7) - 135 + ((amax16 & 0x7Fu) > 0x60u ? 1 : 0);
+  return amax16 == 0u ? 0 : max(e, -127);
+}
+
+// Four bf16 (two words) times s -> four E4M3 codes, element 0 in the low byte.  The
+// product by a power of two is exact except below 2^-126, where E4M3 rounds to +-0
+// either way.
 __device__ __forceinline__ uint32_t encode4(uint32_t a, uint32_t b, float s) {
-  // a, b: two bf16x2 words (elements 0,1 and 2,3) -> 4 codes, element 0 in the low byte
-  const float f0 = __uint_as_float(a << 16) * s, f1 = __uint_as_float(a & 0xFFFF0000u) * s;
-  const float f2 = __uint_as_float(b << 16) * s, f3 = __uint_as_float(b & 0xFFFF0000u) * s;
-  return cvt_e4m3x2_f32(f0, f1) | (cvt_e4m3x2_f32(f2, f3) << 16);
+  float2 p0 = make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+  float2 p1 = make_float2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u));
+  uint64_t r0, r1;
+  const uint64_t ss = ((uint64_t)__float_as_uint(s) << 32) | __float_as_uint(s);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r0) : "l"(*reinterpret_cast<uint64_t*>(&p0)), "l"(ss));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r1) : "l"(*reinterpret_cast<uint64_t*>(&p1)), "l"(ss));
+  const uint32_t c01 = cvt_e4m3x2_f32(__uint_as_float((uint32_t)r0), __uint_as_float((uint32_t)(r0 >> 32)));
+  const uint32_t c23 = cvt_e4m3x2_f32(__uint_as_float((uint32_t)r1), __uint_as_float((uint32_t)(r1 >> 32)));
+  return __byte_perm(c01, c23, 0x5410);
 }
 
 // limit_rows (optional, device): only the first limit_rows[0] * tiles_per_row tiles are
 // processed (the valid rows of a grouped buffer, known only on the device).
+// Lane l of a warp serves tile 4*slot + l/8; its 16 elements are 8 from each half of
+// the tile (16-byte chunk l%8 of bytes 0..127 and of bytes 128..255), so each load
+// instruction reads whole 128-byte lines and each store writes 64 contiguous bytes.
 __global__ void __launch_bounds__(kQThreads) quantize_tiles_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
                                                                     uint8_t* __restrict__ sf, int64_t n_tiles,
                                                                     const int32_t* __restrict__ limit_rows,
@@ -45,27 +66,32 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiles_kernel(const uint4* 
     n_tiles = lim <= 0 ? 0 : min(n_tiles, lim * tiles_per_row);
   }
   const int lane = threadIdx.x & 31;
-  const int sub = lane & 15;  // 16-byte chunk within the tile
+  const int sub = lane & 7;
   const int64_t warp = ((int64_t)blockIdx.x * kQThreads + threadIdx.x) >> 5;
   int64_t tile[kQUnroll];
-  uint4 v[kQUnroll];
+  uint4 v0[kQUnroll], v1[kQUnroll];
 #pragma unroll
   for (int u = 0; u < kQUnroll; ++u) {
-    tile[u] = (warp * kQUnroll + u) * 2 + (lane >> 4);
-    v[u] = tile[u] < n_tiles ? ld_stream(x + tile[u] * 16 + sub) : make_uint4(0u, 0u, 0u, 0u);
+    tile[u] = (warp * kQUnroll + u) * kTilesPerWarp + (lane >> 3);
+    if (tile[u] < n_tiles) {
+      v0[u] = ld_stream(x + tile[u] * 16 + sub);
+      v1[u] = ld_stream(x + tile[u] * 16 + 8 + sub);
+    } else {
+      v0[u] = v1[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 #pragma unroll
   for (int u = 0; u < kQUnroll; ++u) {
-    uint32_t m = absmax8_bits(v[u]);
+    uint32_t m = maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(v0[u].x, v0[u].y), maxabs_bf16x2(v0[u].z, v0[u].w)),
+                               maxabs_bf16x2(maxabs_bf16x2(v1[u].x, v1[u].y), maxabs_bf16x2(v1[u].z, v1[u].w)));
+    m = maxabs_bf16x2(m, __byte_perm(m, 0u, 0x1032)) & 0x7FFFu;
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const int e = tile_exponent(__uint_as_float(m));
-    const float s = exp2_neg(e);  // x * 2^-e is exact (or rounds to +-0 in E4M3 anyway)
+    for (int o = 4; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const int e = bf16_tile_exponent(m);
+    const float s = exp2_neg(e);
     if (tile[u] < n_tiles) {
-      uint2 out;
-      out.x = encode4(v[u].x, v[u].y, s);
-      out.y = encode4(v[u].z, v[u].w, s);
-      q[tile[u] * 16 + sub] = out;
+      q[tile[u] * 16 + sub] = make_uint2(encode4(v0[u].x, v0[u].y, s), encode4(v0[u].z, v0[u].w, s));
+      q[tile[u] * 16 + 8 + sub] = make_uint2(encode4(v1[u].x, v1[u].y, s), encode4(v1[u].z, v1[u].w, s));
       if (sub == 0) sf[tile[u]] = (uint8_t)(e + 127);
     }
   }
@@ -76,7 +102,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiles_kernel(const uint4* 
 cudaError_t launch_quantize_tiles(const void* x, int64_t n_tiles, uint8_t* q, uint8_t* sf, cudaStream_t stream,
                                   const int32_t* limit_rows, int64_t tiles_per_row) {
   if (n_tiles <= 0) return cudaSuccess;
-  const int64_t tiles_per_block = (kQThreads / 32) * kQUnroll * 2;
+  const int64_t tiles_per_block = (kQThreads / 32) * kQUnroll * kTilesPerWarp;
   const int64_t blocks = (n_tiles + tiles_per_block - 1) / tiles_per_block;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
   quantize_tiles_kernel<<<(unsigned)blocks, kQThreads, 0, stream>>>(static_cast<const uint4*>(x),
