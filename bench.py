@@ -480,15 +480,30 @@ def run_profile(args):
     import scaling_aware_transpose_b200 as sat
     from scaling_aware_transpose_b200 import synthetic
     torch.cuda.set_device(0)
-    x = synthetic.to_torch_bf16(synthetic.dense(seed=0)["x"]).cuda()
-    q, sf = sat.quantize_rowwise(x)
-    qt, sft = sat.direct_transpose(q, sf)
-    ws = torch.empty(sat.fp8q_naive_workspace_bytes(ROWS, COLS), dtype=torch.uint8, device="cuda")
-    calls = {
-        "quantize": lambda: sat.fp8q_quantize_rowwise(x, ROWS, COLS, q, sf),
-        "direct": lambda: sat.fp8q_direct_transpose(q, sf, ROWS, COLS, None, 1, qt, sft),
-        "naive": lambda: sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, ws, ws.numel()),
-    }
+    if args.profile in ("quantize", "direct", "naive"):
+        x = synthetic.to_torch_bf16(synthetic.dense(seed=0)["x"]).cuda()
+        q, sf = sat.quantize_rowwise(x)
+        qt, sft = sat.direct_transpose(q, sf)
+        ws = torch.empty(sat.fp8q_naive_workspace_bytes(ROWS, COLS), dtype=torch.uint8, device="cuda")
+        calls = {
+            "quantize": lambda: sat.fp8q_quantize_rowwise(x, ROWS, COLS, q, sf),
+            "direct": lambda: sat.fp8q_direct_transpose(q, sf, ROWS, COLS, None, 1, qt, sft),
+            "naive": lambda: sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, ws, ws.numel()),
+        }
+    elif args.profile == "swiglu":
+        d = synthetic.swiglu()
+        g, u = synthetic.to_torch_bf16(d["gate"]).cuda(), synthetic.to_torch_bf16(d["up"]).cuda()
+        R, C = g.shape
+        q = torch.empty((R, C), dtype=torch.uint8, device="cuda")
+        sf = torch.empty((R, C // 128), dtype=torch.uint8, device="cuda")
+        qt = torch.empty((C, R), dtype=torch.uint8, device="cuda")
+        sft = torch.empty((C, R // 128), dtype=torch.uint8, device="cuda")
+        calls = {"swiglu": lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, qt, sft)}
+    else:  # permute
+        d = synthetic.moe()
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        calls = {"permute": lambda: sat.permute_pad_quant(x, idx, d["num_experts"], 128)}
     torch.cuda.synchronize()
     for _ in range(args.warmup + args.steps):
         calls[args.profile]()
@@ -508,7 +523,7 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true", help="skip the SwiGLU / MoE / stress workload timings")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
-    ap.add_argument("--profile", choices=["quantize", "direct", "naive"], default=None,
+    ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute"], default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)
     if args.profile:

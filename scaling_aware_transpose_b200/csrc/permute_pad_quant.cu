@@ -43,57 +43,85 @@ __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ 
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
-// One CTA: totals, padded exclusive scan into expert offsets, per-chunk bases.
+// Inclusive warp scan of v.
+__device__ __forceinline__ int64_t warp_incl_scan(int64_t v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+// One CTA of 1024 threads (32 warps):
+//  (1) warp w sums expert e's counts over the chunks (e = w, w + 32, ...) -> totals[e];
+//  (2) block-wide exclusive scan of the padded sizes ceil(total/align)*align -> offsets;
+//  (3) warp per expert again: exclusive scan over the chunks -> bases[c][e].
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int64_t C, int E, int align,
                                                     int32_t* __restrict__ offsets, int32_t* __restrict__ bases,
                                                     int32_t* __restrict__ totals) {
   __shared__ int64_t part[1024];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = warp; e < E; e += 32) {
+    int64_t acc = 0;
+    for (int64_t c = lane; c < C; c += 32) acc += counts[c * E + e];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if (lane == 0) totals[e] = (int32_t)acc;
+  }
+  __syncthreads();
   // thread tid owns experts [tid*per, (tid+1)*per)
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
   int64_t local = 0;
-  for (int e = e0; e < e1; ++e) {
-    int64_t tot = 0;
-    for (int64_t c = 0; c < C; ++c) tot += counts[c * E + e];
-    totals[e] = (int32_t)tot;
-    local += (tot + align - 1) / align * align;
-  }
+  for (int e = e0; e < e1; ++e) local += ((int64_t)totals[e] + align - 1) / align * align;
   part[tid] = local;
   __syncthreads();
-  // inclusive scan of part[] (Hillis-Steele)
-  for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+  for (int o = 1; o < (int)blockDim.x; o <<= 1) {  // inclusive scan (Hillis-Steele)
     const int64_t v = tid >= o ? part[tid - o] : 0;
     __syncthreads();
     part[tid] += v;
     __syncthreads();
   }
-  int64_t run = part[tid] - local;  // exclusive prefix of this thread's experts
+  int64_t run = part[tid] - local;
   for (int e = e0; e < e1; ++e) {
     offsets[e] = (int32_t)run;
-    int64_t base = run;
-    for (int64_t c = 0; c < C; ++c) {
-      bases[c * E + e] = (int32_t)base;
-      base += counts[c * E + e];
-    }
-    const int64_t tot = totals[e];
-    run += (tot + align - 1) / align * align;
+    run += ((int64_t)totals[e] + align - 1) / align * align;
   }
   if (tid == blockDim.x - 1) offsets[E] = (int32_t)part[tid];
+  __syncthreads();
+  for (int e = warp; e < E; e += 32) {
+    int64_t carry = offsets[e];
+    for (int64_t c0 = 0; c0 < C; c0 += 32) {
+      const int64_t c = c0 + lane;
+      const int64_t v = c < C ? counts[c * E + e] : 0;
+      const int64_t incl = warp_incl_scan(v, lane);
+      if (c < C) bases[c * E + e] = (int32_t)(carry + incl - v);
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+  }
 }
 
-// One warp per chunk: stable destination rows in (t, s) order.
+// One warp per chunk: stable destination rows in (t, s) order.  The chunk's routing ids
+// are loaded up front so that the 32 ranking steps do not wait on memory.
 __global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
                                                   const int32_t* __restrict__ bases, int32_t* __restrict__ row_id_map) {
   extern __shared__ int32_t run[];
   const int lane = threadIdx.x;
+  const int64_t p0 = (int64_t)blockIdx.x * kChunk;
+  int32_t ids[kChunk / 32];
+#pragma unroll
+  for (int i = 0; i < kChunk / 32; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    ids[i] = p < npairs ? __ldg(idx + p) : -1;
+  }
   for (int e = lane; e < E; e += 32) run[e] = bases[(int64_t)blockIdx.x * E + e];
   __syncwarp();
-  const int64_t p0 = (int64_t)blockIdx.x * kChunk;
-  for (int i = 0; i < kChunk; i += 32) {
-    const int64_t p = p0 + i + lane;
+#pragma unroll 4
+  for (int i = 0; i < kChunk / 32; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
     const bool live = p < npairs;
-    const int32_t e = live ? __ldg(idx + p) : -1;
+    const int32_t e = ids[i];
     const bool ok = live && e >= 0 && e < E;
     const int32_t key = ok ? e : -1 - lane;  // invalid lanes never match anyone
     const unsigned same = __match_any_sync(0xFFFFFFFFu, key);
@@ -110,52 +138,67 @@ __global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ id
   }
 }
 
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4& v) {
-  const uint32_t m0 = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-  const uint32_t m1 = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
-  const uint32_t m = __vmaxu2(m0, m1);
-  return max(m & 0xFFFFu, m >> 16) << 16;
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// Tile exponent from the BF16 amax bit pattern (see quantize_rowwise.cu): e = E - 135,
+// plus one when the mantissa exceeds 0x60; 0 for a zero tile; clamped at -127.
+__device__ __forceinline__ int bf16_tile_exponent(uint32_t amax16) {
+  const int e = (int)(amax16 >> 7) - 135 + ((amax16 & 0x7Fu) > 0x60u ? 1 : 0);
+  return amax16 == 0u ? 0 : max(e, -127);
 }
 __device__ __forceinline__ uint32_t encode4(uint32_t a, uint32_t b, float s) {
   const float f0 = __uint_as_float(a << 16) * s, f1 = __uint_as_float(a & 0xFFFF0000u) * s;
   const float f2 = __uint_as_float(b << 16) * s, f3 = __uint_as_float(b & 0xFFFF0000u) * s;
-  return cvt_e4m3x2_f32(f0, f1) | (cvt_e4m3x2_f32(f2, f3) << 16);
+  return __byte_perm(cvt_e4m3x2_f32(f0, f1), cvt_e4m3x2_f32(f2, f3), 0x5410);
 }
 
 constexpr int kSThreads = 256;
-constexpr int kSUnroll = 4;
+constexpr int kSUnroll = 2;
 
-// Tiles of x (token t, column block j) in row-major order; 16 lanes per tile.
+// Tiles of x (token t, column block j) in row-major order: 8 lanes per tile, 16 bf16 per
+// lane (8 from each half of the tile), four tiles per warp per slot.  Each tile is read
+// and quantized once and its codes written to the token's top-k destination rows.
 __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* __restrict__ x, int64_t tokens, int ncb,
                                                                   const int32_t* __restrict__ row_id_map, int topk,
                                                                   uint2* __restrict__ q, uint8_t* __restrict__ sf) {
-  const int lane = threadIdx.x & 31, sub = lane & 15;
+  const int lane = threadIdx.x & 31, sub = lane & 7;
   const int64_t n_tiles = tokens * ncb;
   const int64_t warp = ((int64_t)blockIdx.x * kSThreads + threadIdx.x) >> 5;
   int64_t tile[kSUnroll];
-  uint4 v[kSUnroll];
+  uint4 v0[kSUnroll], v1[kSUnroll];
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
-    tile[u] = (warp * kSUnroll + u) * 2 + (lane >> 4);
-    v[u] = tile[u] < n_tiles ? ld_stream(x + tile[u] * 16 + sub) : make_uint4(0u, 0u, 0u, 0u);
+    tile[u] = (warp * kSUnroll + u) * 4 + (lane >> 3);
+    if (tile[u] < n_tiles) {
+      v0[u] = ld_stream(x + tile[u] * 16 + sub);
+      v1[u] = ld_stream(x + tile[u] * 16 + 8 + sub);
+    } else {
+      v0[u] = v1[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
-    uint32_t m = absmax8_bits(v[u]);
+    uint32_t m = maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(v0[u].x, v0[u].y), maxabs_bf16x2(v0[u].z, v0[u].w)),
+                               maxabs_bf16x2(maxabs_bf16x2(v1[u].x, v1[u].y), maxabs_bf16x2(v1[u].z, v1[u].w)));
+    m = maxabs_bf16x2(m, __byte_perm(m, 0u, 0x1032)) & 0x7FFFu;
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    for (int o = 4; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if (tile[u] >= n_tiles) continue;
-    const int e = tile_exponent(__uint_as_float(m));
+    const int e = bf16_tile_exponent(m);
     const float s = exp2_neg(e);
-    uint2 out;
-    out.x = encode4(v[u].x, v[u].y, s);
-    out.y = encode4(v[u].z, v[u].w, s);
+    const uint2 lo = make_uint2(encode4(v0[u].x, v0[u].y, s), encode4(v0[u].z, v0[u].w, s));
+    const uint2 hi = make_uint2(encode4(v1[u].x, v1[u].y, s), encode4(v1[u].z, v1[u].w, s));
     const int64_t t = tile[u] / ncb;
     const int j = (int)(tile[u] - t * ncb);
     for (int k = 0; k < topk; ++k) {
       const int32_t row = __ldg(row_id_map + t * topk + k);
       if (row < 0) continue;
-      q[((int64_t)row * ncb + j) * 16 + sub] = out;
+      uint2* dst = q + ((int64_t)row * ncb + j) * 16;
+      dst[sub] = lo;
+      dst[8 + sub] = hi;
       if (sub == 0) sf[(int64_t)row * ncb + j] = (uint8_t)(e + 127);
     }
   }
@@ -210,7 +253,7 @@ fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64
   if (hidden == 0) return FP8Q_OK;  // routing only: offsets and row ids, no payload
   const int ncb = (int)(hidden / 128);
   const int64_t n_tiles = tokens * ncb;
-  const int64_t tiles_per_block = (kSThreads / 32) * kSUnroll * 2;
+  const int64_t tiles_per_block = (kSThreads / 32) * kSUnroll * 4;
   scatter_quant_kernel<<<(unsigned)((n_tiles + tiles_per_block - 1) / tiles_per_block), kSThreads, 0, stream>>>(
       static_cast<const uint4*>(x), tokens, ncb, row_id_map, topk, reinterpret_cast<uint2*>(q), sf);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;

@@ -11,7 +11,7 @@
 // Arithmetic spec of y (every step one IEEE fp32 operation, round to nearest even, no
 // contraction; identical on every implementation of this spec):
 //   exp(a):  a > 89 -> +inf, a < -104 -> +0; otherwise (Cody & Waite, "Software Manual
-//            for the Elementary Functions", 1980) n = rint(a * L2E),
+//            for the Elementary Functions", 1980) n = rint(a * L2E) (ties to even),
 //            r = fma(-n, LN2_HI, a), r = fma(-n, LN2_LO, r), p = Horner over 1/k!, k=7..0,
 //            result = (p * 2^floor(n/2)) * 2^(n - floor(n/2));
 //   silu(g) = g / (1 + exp(-g));   y = silu(g) * u.
@@ -29,9 +29,14 @@ constexpr float kLn2Lo = 0x1.7f7d1cp-20f;
 constexpr float kC0 = 0x1p+0f, kC1 = 0x1p+0f, kC2 = 0x1p-1f, kC3 = 0x1.555556p-3f;  // 1/k!
 constexpr float kC4 = 0x1.555556p-5f, kC5 = 0x1.111112p-7f, kC6 = 0x1.6c16c2p-10f, kC7 = 0x1.a01a02p-13f;
 
+// rint(t) for |t| < 2^22 is (t + 1.5*2^23) - 1.5*2^23 with both additions rounded to
+// nearest even (the first sum lies in [2^23, 2^24), whose ulp is 1); the integer n is read
+// off the bits of the first sum.  Same result as rintf, without the conversion unit.
 __device__ __forceinline__ float exp_spec(float a) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   const float ac = fminf(fmaxf(a, -104.0f), 89.0f);  // keeps n in [-150, 128]
-  const float n = rintf(__fmul_rn(ac, kL2E));
+  const float tm = __fadd_rn(__fmul_rn(ac, kL2E), kMagic);
+  const float n = __fadd_rn(tm, -kMagic);
   float r = __fmaf_rn(-n, kLn2Hi, ac);
   r = __fmaf_rn(-n, kLn2Lo, r);
   float p = kC7;
@@ -42,7 +47,7 @@ __device__ __forceinline__ float exp_spec(float a) {
   p = __fmaf_rn(p, r, kC2);
   p = __fmaf_rn(p, r, kC1);
   p = __fmaf_rn(p, r, kC0);
-  const int ni = (int)n;
+  const int ni = __float_as_int(tm) - 0x4B400000;
   const int n1 = ni >> 1;  // floor(n / 2)
   const int n2 = ni - n1;
   const float res = __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
@@ -59,7 +64,7 @@ constexpr int kPasses = 4;  // 4 passes x 32 rows x (8 threads x 16 elements)
 
 __device__ __forceinline__ uint32_t swizzled_chunk(int row, int chunk) { return (uint32_t)(chunk ^ ((row >> 2) & 7)); }
 
-__global__ void __launch_bounds__(kThreads) swiglu_quant_kernel(const uint16_t* __restrict__ gate,
+__global__ void __launch_bounds__(kThreads, 3) swiglu_quant_kernel(const uint16_t* __restrict__ gate,
                                                                 const uint16_t* __restrict__ up, int64_t rows, int cols,
                                                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                                                                 uint8_t* __restrict__ qt, uint8_t* __restrict__ sft) {
