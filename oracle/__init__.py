@@ -54,6 +54,8 @@ def _declare(L):
         "orc_exp_spec_constants": [V],
         "orc_exp_spec_array": [V, I64, V],
         "orc_swiglu_array": [V, V, I64, V],
+        "orc_pack_ue8m0": [V, I64, I64, V],
+        "orc_quantize_rowwise_opt": [V, I64, I64, ctypes.c_int, V, V],
     }.items():
         fn = getattr(L, name)
         fn.argtypes, fn.restype = args, None
@@ -62,6 +64,7 @@ def _declare(L):
         "orc_naive_transpose": [V, V, I64, I64, V, I32, V, V],
         "orc_swiglu_quant": [V, V, I64, I64, V, V, V, V],
         "orc_permute_pad_quant": [V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
+        "orc_quantize_rowwise_colwise": [V, I64, I64, ctypes.c_uint32, V, V, V, V],
     }.items():
         fn = getattr(L, name)
         fn.argtypes, fn.restype = args, ctypes.c_int
@@ -125,6 +128,55 @@ def quantize_rowwise_f32(y):
     sf = np.empty((rows, cols // 128), np.uint8)
     lib().orc_quantize_rowwise_f32(_p(y), rows, cols, _p(q), _p(sf))
     return q, sf
+
+
+ZERO_TILE_MIN_SCALE = 1  # flags of the single-pass quantizer (same meaning as the library's)
+SF_PACKED_UE8M0 = 2
+
+
+def packed_sf_shape(mn: int, ktiles: int) -> tuple[int, int]:
+    """Shape (words) of the packed UE8M0 scales of an operand with mn rows and ktiles
+    1x128 tiles along K."""
+    return ((ktiles + 3) // 4, (mn + 3) // 4 * 4)
+
+
+def pack_ue8m0(sf):
+    """Unpacked scale bytes [mn, ktiles] -> packed words [ceil(ktiles/4), mn_pad] (uint32)."""
+    sf = _c(sf, np.uint8)
+    mn, kt = sf.shape
+    out = np.empty(packed_sf_shape(mn, kt), np.uint32)
+    lib().orc_pack_ue8m0(_p(sf), mn, kt, _p(out))
+    return out
+
+
+def quantize_rowwise_opt(x_bf16_bits, zero_tile_min: bool):
+    x = _c(x_bf16_bits, np.uint16)
+    rows, cols = x.shape
+    if cols % 128:
+        raise OracleError("cols must be a multiple of 128")
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // 128), np.uint8)
+    lib().orc_quantize_rowwise_opt(_p(x), rows, cols, 1 if zero_tile_min else 0, _p(q), _p(sf))
+    return q, sf
+
+
+def quantize_rowwise_colwise(x_bf16_bits, flags: int = 0, colwise: bool = True):
+    """Single-pass quantizer's definition: (Q, SF, Q^T, SF^T); Q^T/SF^T are None when
+    colwise is False.  With SF_PACKED_UE8M0 the scales are packed uint32 words."""
+    x = _c(x_bf16_bits, np.uint16)
+    rows, cols = x.shape
+    packed = bool(flags & SF_PACKED_UE8M0)
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty(packed_sf_shape(rows, cols // 128), np.uint32) if packed else np.empty((rows, cols // 128), np.uint8)
+    qt = sft = None
+    if colwise:
+        qt = np.empty((cols, rows), np.uint8)
+        sft = (np.empty(packed_sf_shape(cols, rows // 128), np.uint32) if packed
+               else np.empty((cols, rows // 128), np.uint8))
+    rc = lib().orc_quantize_rowwise_colwise(_p(x), rows, cols, int(flags), _p(q), _p(sf), _p(qt), _p(sft))
+    if rc:
+        raise OracleError(f"oracle single-pass quantizer rejected its arguments (code {rc})")
+    return q, sf, qt, sft
 
 
 def _transpose_common(fn, q, sf, offsets):

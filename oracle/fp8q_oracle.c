@@ -211,8 +211,10 @@ void orc_shift_codes(const uint8_t *c, int64_t n, int k, int bytes_rule, uint8_t
 /* Row-wise 1x128 quantization ([DSV3] §3; [FLOW] 一句话总结/核心方法)  */
 /* ------------------------------------------------------------------ */
 
-/* One 1x128 tile given as exact doubles: amax, e, codes. */
-static void quantize_tile(const double *v, uint8_t *q, uint8_t *sf)
+/* One 1x128 tile given as exact doubles: amax, e, codes.  zero_e is the exponent an
+ * all-zero tile takes: 0 by the pages' rule (S = 1), or -127 under the zero-tile option
+ * of the single-pass quantizer (below). */
+static void quantize_tile_z(const double *v, int zero_e, uint8_t *q, uint8_t *sf)
 {
     double amax = 0.0;
     for (int i = 0; i < 128; i++) {
@@ -220,11 +222,13 @@ static void quantize_tile(const double *v, uint8_t *q, uint8_t *sf)
         if (a > amax)
             amax = a;
     }
-    int e = orc_scale_exponent(amax);
+    int e = amax == 0.0 ? zero_e : orc_scale_exponent(amax);
     for (int i = 0; i < 128; i++)
         q[i] = orc_e4m3_encode(ldexp(v[i], -e)); /* x * 2^-e is exact in double */
     *sf = (uint8_t)(e + 127);                        /* UE8M0 byte, bias 127 */
 }
+
+static void quantize_tile(const double *v, uint8_t *q, uint8_t *sf) { quantize_tile_z(v, 0, q, sf); }
 
 /* X bf16 [rows, cols] (cols % 128 == 0) -> Q u8 [rows, cols], SF u8 [rows, cols/128]. */
 void orc_quantize_rowwise(const uint16_t *x, int64_t rows, int64_t cols, uint8_t *q, uint8_t *sf)
@@ -397,6 +401,92 @@ int orc_naive_transpose(const uint8_t *q, const uint8_t *sf, int64_t rows, int64
     free(v);
     free(vt);
     return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Single-pass quantization into both layouts, packed UE8M0 scales      */
+/* ------------------------------------------------------------------ */
+
+/* Packed UE8M0 ([DSV3] §8: the SM100 GEMM takes power-of-two scales four to a 32-bit
+ * word, each byte being the exponent byte of the fp32 scale, i.e. e + 127).
+ * Input: unpacked scales sf [mn, ktiles] (one byte per 1x128 tile along K).
+ * Output: words [ceil(ktiles/4), mn_pad], MN-major, word (g, m) at index g*mn_pad + m,
+ * holding the scale of K tile 4g+i in byte i (bits 8i..8i+7).
+ * Readings (the pages give only "four 8-bit scales in one int32"): bytes in K order
+ * from the least significant end; MN-major so that a GEMM tile of consecutive rows
+ * reads consecutive words; mn padded up to a multiple of 4 (16-byte rows); bytes of K
+ * tiles past the last one, and words of padding rows, are 0. */
+void orc_pack_ue8m0(const uint8_t *sf, int64_t mn, int64_t ktiles, uint32_t *out)
+{
+    int64_t groups = (ktiles + 3) / 4;
+    int64_t mn_pad = (mn + 3) / 4 * 4;
+    for (int64_t g = 0; g < groups; g++)
+        for (int64_t m = 0; m < mn_pad; m++) {
+            uint32_t w = 0;
+            for (int i = 0; i < 4; i++) {
+                int64_t kt = 4 * g + i;
+                if (m < mn && kt < ktiles)
+                    w |= (uint32_t)sf[m * ktiles + kt] << (8 * i);
+            }
+            out[g * mn_pad + m] = w;
+        }
+}
+
+/* Row-wise quantization with the zero-tile option: zero_tile_min != 0 gives an
+ * all-zero tile e = -127 (scale byte 0x00) instead of e = 0.  Reading: the pages fix
+ * S = 1 for a zero tile, which lets zero rows (padding, dead tokens) raise a block's
+ * Smax in the direct transpose and push the other rows' small values toward zero; the
+ * option (ours, off by default) gives such tiles the smallest scale, so Smax is the max
+ * over the nonzero tiles.  The codes of a zero tile are +-0 either way. */
+void orc_quantize_rowwise_opt(const uint16_t *x, int64_t rows, int64_t cols, int zero_tile_min, uint8_t *q,
+                              uint8_t *sf)
+{
+    int64_t nt = cols / 128;
+    int zero_e = zero_tile_min ? -127 : 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < rows; t++) {
+        double v[128];
+        for (int64_t j = 0; j < nt; j++) {
+            for (int i = 0; i < 128; i++)
+                v[i] = bf16_to_double(x[t * cols + j * 128 + i]);
+            quantize_tile_z(v, zero_e, q + t * cols + j * 128, sf + t * nt + j);
+        }
+    }
+}
+
+/* BF16 X [rows, cols] -> the row-wise (Q, SF) and, when qt is non-NULL, the
+ * column-wise (Q^T, SF^T) layouts: by definition the row-wise quantization followed by
+ * the scaling-aware direct transpose of its result ([FLOW] 核心方法).  flags bit 0:
+ * zero-tile option; bit 1: scales written packed (orc_pack_ue8m0) - sf as
+ * [ceil(cols/512), rows] words, sft as [ceil(rows/512), cols] words - instead of bytes
+ * [rows, cols/128] and [cols, rows/128].  Returns 0, 2 (shape), 5 (allocation). */
+int orc_quantize_rowwise_colwise(const uint16_t *x, int64_t rows, int64_t cols, uint32_t flags, uint8_t *q,
+                                 void *sf, uint8_t *qt, void *sft)
+{
+    if (cols % 128 || (qt && rows % 128))
+        return 2;
+    int packed = (flags & 2u) != 0;
+    uint8_t *sf_b = packed ? (uint8_t *)malloc((size_t)(rows * cols / 128)) : (uint8_t *)sf;
+    uint8_t *sft_b = (packed && qt) ? (uint8_t *)malloc((size_t)(rows * cols / 128)) : (uint8_t *)sft;
+    if (!sf_b || (qt && !sft_b)) {
+        if (packed) {
+            free(sf_b);
+            free(sft_b);
+        }
+        return 5;
+    }
+    orc_quantize_rowwise_opt(x, rows, cols, (int)(flags & 1u), q, sf_b);
+    int rc = 0;
+    if (qt)
+        rc = orc_direct_transpose(q, sf_b, rows, cols, NULL, 1, qt, sft_b);
+    if (packed) {
+        orc_pack_ue8m0(sf_b, rows, cols / 128, (uint32_t *)sf);
+        if (qt)
+            orc_pack_ue8m0(sft_b, cols, rows / 128, (uint32_t *)sft);
+        free(sf_b);
+        free(sft_b);
+    }
+    return rc;
 }
 
 /* ------------------------------------------------------------------ */
