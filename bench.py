@@ -37,6 +37,7 @@ N_ELEM = ROWS * COLS
 BYTES_QUANT = 2 * N_ELEM + N_ELEM + N_ELEM // 128            # read X, write Q + SF
 BYTES_DIRECT = N_ELEM + N_ELEM // 128 + N_ELEM + N_ELEM // 128  # read Q + SF, write Q^T + SF^T
 BYTES_STEP = BYTES_QUANT + BYTES_DIRECT
+BYTES_ROWCOL = 2 * N_ELEM + 2 * (N_ELEM + N_ELEM // 128)      # read X, write Q + SF + Q^T + SF^T
 METRIC = "direct-transpose & quantize GB/s on 1 B200 (% of HBM peak); bit-exact vs oracle"
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
@@ -56,7 +57,7 @@ def measured_peak_gbs():
 def kernel_sources(kind: str):
     csrc = os.path.join(ROOT, "scaling_aware_transpose_b200", "csrc")
     main = {"quantize": "quantize_rowwise.cu", "direct": "direct_transpose.cu", "swiglu": "swiglu_quant.cu",
-            "permute": "permute_pad_quant.cu"}[kind]
+            "permute": "permute_pad_quant.cu", "rowwise_colwise": "quantize_rowwise_colwise.cu"}[kind]
     return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")]
 
 
@@ -71,7 +72,8 @@ def source_digest(paths) -> str:
 def profiled_traffic(kind: str):
     """DRAM bytes per launch from the committed ncu summary of this kernel on this
     workload, or None when there is none or the kernel source changed since."""
-    name = {"quantize": "quantize_rowwise_dense_8192x7168.md", "direct": "direct_transpose_dense_8192x7168.md"}[kind]
+    name = {"quantize": "quantize_rowwise_dense_8192x7168.md", "direct": "direct_transpose_dense_8192x7168.md",
+            "rowwise_colwise": "quantize_rowwise_colwise_dense_8192x7168.md"}[kind]
     p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
@@ -368,6 +370,22 @@ def run_ours(args, rank, world, local_rank):
     t_q_clean = time_on_stream(quant, min(K, 50), stream, clean_flush)
     t_d_clean = time_on_stream(direct, min(K, 50), stream, clean_flush)
 
+    # single-pass quantizer: the same four outputs from one read of X (byte-identical to
+    # the two-kernel step); also with packed UE8M0 scales and the zero-tile option
+    rc_q, rc_sf = torch.empty_like(q), torch.empty_like(sf)
+    rc_qt, rc_sft = torch.empty_like(qt), torch.empty_like(sft)
+    pk_sf = torch.empty(sat.packed_sf_shape(ROWS, COLS), dtype=torch.int32, device=device)
+    pk_sft = torch.empty(sat.packed_sf_shape(COLS, ROWS), dtype=torch.int32, device=device)
+    rowcol = lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, 0, rc_q, rc_sf, rc_qt, rc_sft, sp)
+    rowcol_pk = lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, sat.ZERO_TILE_MIN_SCALE |
+                                                          sat.SF_PACKED_UE8M0, rc_q, pk_sf, rc_qt, pk_sft, sp)
+    t_rc = time_on_stream(rowcol, min(K, 50) + 3, stream, lambda: flush.fill_(10))
+    t_rc_clean = time_on_stream(rowcol, min(K, 50) + 3, stream, clean_flush)
+    t_rc_pk = time_on_stream(rowcol_pk, min(K, 50) + 3, stream, lambda: flush.fill_(11))
+    rowcol()
+    torch.cuda.synchronize()
+    same_rc = all(torch.equal(a_, b_) for a_, b_ in ((rc_q, q), (rc_sf, sf), (rc_qt, qt), (rc_sft, sft)))
+
     # ---- end to end through the C ABI from pinned host buffers
     q_h = torch.empty_like(q, device="cpu").pin_memory()
     sf_h = torch.empty_like(sf, device="cpu").pin_memory()
@@ -423,6 +441,16 @@ def run_ours(args, rank, world, local_rank):
                                       "direct_speedup": round(t_naive / avg_d, 2)},
             "chained_step_no_flush_between": {"us": round(t_chain * 1e6, 2),
                                               "GB/s": round(BYTES_STEP / t_chain / 1e9, 1)},
+            "quantize_rowwise_colwise_single_pass": {
+                "us": round(t_rc * 1e6, 2), "bytes": BYTES_ROWCOL, "GB/s": round(BYTES_ROWCOL / t_rc / 1e9, 1),
+                "frac_of_peak": round(BYTES_ROWCOL / t_rc / 1e9 / peak, 4),
+                "frac_of_8000": round(BYTES_ROWCOL / t_rc / 1e9 / 8000, 4),
+                "clean_l2_us": round(t_rc_clean * 1e6, 2),
+                "clean_l2_GB/s": round(BYTES_ROWCOL / t_rc_clean / 1e9, 1),
+                "packed_ue8m0_zero_tile_us": round(t_rc_pk * 1e6, 2),
+                "vs_two_kernel_step": round((avg_q + avg_d) / t_rc, 3),
+                "outputs_equal_two_kernel_step": same_rc,
+                "traffic": profiled_traffic("rowwise_colwise")},
             "clean_l2_flush": {"quantize_us": round(t_q_clean * 1e6, 2),
                                "quantize_GB/s": round(BYTES_QUANT / t_q_clean / 1e9, 1),
                                "direct_us": round(t_d_clean * 1e6, 2),
@@ -481,7 +509,7 @@ def run_profile(args):
     import scaling_aware_transpose_b200 as sat
     from scaling_aware_transpose_b200 import synthetic
     torch.cuda.set_device(0)
-    if args.profile in ("quantize", "direct", "naive"):
+    if args.profile in ("quantize", "direct", "naive", "rowwise_colwise"):
         x = synthetic.to_torch_bf16(synthetic.dense(seed=0)["x"]).cuda()
         q, sf = sat.quantize_rowwise(x)
         qt, sft = sat.direct_transpose(q, sf)
@@ -490,6 +518,7 @@ def run_profile(args):
             "quantize": lambda: sat.fp8q_quantize_rowwise(x, ROWS, COLS, q, sf),
             "direct": lambda: sat.fp8q_direct_transpose(q, sf, ROWS, COLS, None, 1, qt, sft),
             "naive": lambda: sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, ws, ws.numel()),
+            "rowwise_colwise": lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, 0, q, sf, qt, sft),
         }
     elif args.profile == "swiglu":
         d = synthetic.swiglu()
@@ -524,7 +553,8 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true", help="skip the SwiGLU / MoE / stress workload timings")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
-    ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute"], default=None,
+    ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise"],
+                    default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)
     if args.profile:

@@ -153,6 +153,43 @@ fp8q_status fp8q_permute_pad_quant(const void *x, int64_t tokens, int64_t hidden
                                    int32_t *row_id_map, void *workspace, size_t workspace_bytes,
                                    fp8q_stream_t stream);
 
+/* Options of fp8q_quantize_rowwise_colwise (bit flags). */
+#define FP8Q_ZERO_TILE_MIN_SCALE 0x1u /* all-zero tiles take e = -127 (byte 0x00), not e = 0 */
+#define FP8Q_SF_PACKED_UE8M0 0x2u     /* scales as packed UE8M0 words (see below) */
+
+/* Bytes of a packed UE8M0 scale tensor for an FP8 operand with `mn` rows along M/N and
+ * `k` elements along K (k % 128 == 0): 4 * ceil(k/512) * (mn rounded up to 4).
+ * 0 for non-positive sizes. */
+size_t fp8q_packed_sf_bytes(int64_t mn, int64_t k);
+
+/* Single-pass quantization into both layouts: one read of X produces the row-wise
+ * (Q, SF) of fp8q_quantize_rowwise and the column-wise (Q^T, SF^T) that
+ * fp8q_direct_transpose would make from them - byte for byte the same results
+ * (FP8-Flow-MoE 核心方法; DeepSeek FP8 §1, §3).  Moves 4 bytes per element instead of
+ * the 5 of the two separate calls.
+ *   x   : bf16 [rows, cols], cols % 128 == 0; rows % 128 == 0 when qt is given.
+ *   q   : u8 [rows, cols]   out, as fp8q_quantize_rowwise.
+ *   sf  : out. Unpacked: u8 [rows, cols/128].  Packed: u32 [ceil(cols/512), rows4].
+ *   qt  : u8 [cols, rows] out, or NULL for the row-wise layout only.
+ *   sft : out, NULL iff qt is NULL.  Unpacked: u8 [cols, rows/128] (as the direct
+ *         transpose).  Packed: u32 [ceil(rows/512), cols].
+ *   flags: FP8Q_ZERO_TILE_MIN_SCALE - an all-zero 1x128 tile gets e = -127 instead of
+ *         e = 0, so it never raises Smax of its 128x128 block (its codes are +-0 either
+ *         way; a fully zero block gets SF^T byte 0).  Off, results equal
+ *         fp8q_quantize_rowwise + fp8q_direct_transpose exactly.
+ *         FP8Q_SF_PACKED_UE8M0 - scales as packed UE8M0 (DeepSeek FP8 §8: the SM100 GEMM
+ *         reads four power-of-two scales per int32): word (g, m) at index g*mn4 + m
+ *         (mn4 = mn rounded up to 4; MN-major) holds the scale bytes of the K tiles
+ *         4g..4g+3 of row m in bits 0-7, 8-15, 16-23, 24-31.  Bytes of K tiles past the
+ *         last, and words of the padding rows m >= mn, are 0.  sf/sft must then be
+ *         4-byte aligned and hold fp8q_packed_sf_bytes(rows, cols) and
+ *         fp8q_packed_sf_bytes(cols, rows) bytes.
+ * x, q and qt must be 16-byte aligned.  Errors: NULL, ALIGN, SHAPE, ARG (unknown flag
+ * bits, qt/sft not both NULL or both set), CUDA. */
+fp8q_status fp8q_quantize_rowwise_colwise(const void *x, int64_t rows, int64_t cols, uint32_t flags,
+                                          uint8_t *q, void *sf, uint8_t *qt, void *sft,
+                                          fp8q_stream_t stream);
+
 /* Size of the library's static scratch for fp8q_permute_pad_quant_noalloc (4 MiB). */
 #define FP8Q_NOALLOC_SCRATCH_BYTES (4u << 20)
 

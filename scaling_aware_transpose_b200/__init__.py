@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
             "fp8q_naive_workspace_bytes": ([I64, I64], SZ),
             "fp8q_naive_transpose": ([P, P, I64, I64, P, I32, P, P, P, SZ, P], ctypes.c_int),
             "fp8q_swiglu_quant": ([P, P, I64, I64, P, P, P, P, P], ctypes.c_int),
+            "fp8q_packed_sf_bytes": ([I64, I64], SZ),
+            "fp8q_quantize_rowwise_colwise": ([P, I64, I64, ctypes.c_uint32, P, P, P, P, P], ctypes.c_int),
             "fp8q_permute_workspace_bytes": ([I64, I32, I32], SZ),
             "fp8q_permute_pad_quant": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
             "fp8q_permute_pad_quant_noalloc": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P], ctypes.c_int),
@@ -130,6 +132,19 @@ def fp8q_naive_transpose(q, sf, rows: int, cols: int, group_offsets, num_groups:
 def fp8q_swiglu_quant(gate, up, rows: int, cols: int, q, sf, qt, sft, stream=None) -> None:
     _check(lib().fp8q_swiglu_quant(_ptr(gate), _ptr(up), rows, cols, _ptr(q), _ptr(sf), _ptr(qt), _ptr(sft),
                                    _stream(stream)), "fp8q_swiglu_quant")
+
+
+ZERO_TILE_MIN_SCALE = 0x1  # FP8Q_ZERO_TILE_MIN_SCALE
+SF_PACKED_UE8M0 = 0x2      # FP8Q_SF_PACKED_UE8M0
+
+
+def fp8q_packed_sf_bytes(mn: int, k: int) -> int:
+    return int(lib().fp8q_packed_sf_bytes(mn, k))
+
+
+def fp8q_quantize_rowwise_colwise(x, rows: int, cols: int, flags: int, q, sf, qt, sft, stream=None) -> None:
+    _check(lib().fp8q_quantize_rowwise_colwise(_ptr(x), rows, cols, int(flags), _ptr(q), _ptr(sf), _ptr(qt),
+                                               _ptr(sft), _stream(stream)), "fp8q_quantize_rowwise_colwise")
 
 
 def fp8q_permute_workspace_bytes(tokens: int, topk: int, num_experts: int) -> int:
@@ -224,6 +239,29 @@ def swiglu_quant(gate, up, transposed: bool = True, stream=None):
     qt = _empty((cols, rows), torch.uint8, gate) if transposed else None
     sft = _empty((cols, rows // 128), torch.uint8, gate) if transposed else None
     fp8q_swiglu_quant(gate, up, rows, cols, q, sf, qt, sft, stream)
+    return q, sf, qt, sft
+
+
+def packed_sf_shape(mn: int, k: int) -> tuple[int, int]:
+    """Shape (int32 words) of packed UE8M0 scales for an operand [mn, k]."""
+    return ((k // 128 + 3) // 4, (mn + 3) // 4 * 4)
+
+
+def quantize_rowwise_colwise(x, flags: int = 0, colwise: bool = True, stream=None):
+    """One read of x -> (Q, SF, Q^T, SF^T); Q^T/SF^T are None when colwise is False.
+    With SF_PACKED_UE8M0 the scales are int32 tensors of packed UE8M0 words."""
+    import torch
+    rows, cols = x.shape
+    packed = bool(flags & SF_PACKED_UE8M0)
+    q = _empty((rows, cols), torch.uint8, x)
+    sf = (_empty(packed_sf_shape(rows, cols), torch.int32, x) if packed
+          else _empty((rows, cols // 128), torch.uint8, x))
+    qt = sft = None
+    if colwise:
+        qt = _empty((cols, rows), torch.uint8, x)
+        sft = (_empty(packed_sf_shape(cols, rows), torch.int32, x) if packed
+               else _empty((cols, rows // 128), torch.uint8, x))
+    fp8q_quantize_rowwise_colwise(x, rows, cols, flags, q, sf, qt, sft, stream)
     return q, sf, qt, sft
 
 

@@ -224,18 +224,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 }  // namespace
 
 fp8q_status launch_direct_transpose(const DeviceInfo& dev, const uint8_t* q, const uint8_t* sf, int64_t rows,
@@ -243,7 +231,7 @@ fp8q_status launch_direct_transpose(const DeviceInfo& dev, const uint8_t* q, con
                                     uint8_t* sft, cudaStream_t stream) {
   const int64_t nunits_max = (rows / 128) * (cols / 128) * 2;
   if (nunits_max == 0) return FP8Q_OK;
-  auto encode = get_encoder();
+  auto encode = tensor_map_encoder();
   if (!encode) return FP8Q_ERR_CUDA;
   CUtensorMap map;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};

@@ -33,6 +33,20 @@ fp8q_status device_info(DeviceInfo* out) {
   return FP8Q_OK;
 }
 
+// The driver's tensor-map encoder, fetched through the runtime once (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
 // ---- bounded-wait test hook: one mbarrier nobody arrives at
 __global__ void expire_wait_kernel(uint64_t timeout_ns, int* status) {
   __shared__ uint64_t bar;
@@ -151,6 +165,29 @@ fp8q_status fp8q_swiglu_quant(const void* gate, const void* up, int64_t rows, in
   fp8q::DeviceInfo dev;
   if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
   return fp8q::launch_swiglu_quant(dev, gate, up, rows, cols, q, sf, qt, sft, as_stream(stream));
+}
+
+size_t fp8q_packed_sf_bytes(int64_t mn, int64_t k) {
+  if (mn <= 0 || k <= 0) return 0;
+  return (size_t)(4 * ((k / 128 + 3) / 4) * ((mn + 3) / 4 * 4));
+}
+
+fp8q_status fp8q_quantize_rowwise_colwise(const void* x, int64_t rows, int64_t cols, uint32_t flags, uint8_t* q,
+                                          void* sf, uint8_t* qt, void* sft, fp8q_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 128 || rows > kMaxDim || cols > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (flags & ~(FP8Q_ZERO_TILE_MIN_SCALE | FP8Q_SF_PACKED_UE8M0)) return FP8Q_ERR_ARG;
+  if ((qt == nullptr) != (sft == nullptr)) return FP8Q_ERR_ARG;
+  if (qt && rows % 128) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  if (!x || !q || !sf) return FP8Q_ERR_NULL;
+  const bool packed = (flags & FP8Q_SF_PACKED_UE8M0) != 0;
+  const uintptr_t sf_mask = packed ? 3u : 0u;
+  if (!aligned16(x) || !aligned16(q) || (qt && !aligned16(qt)) || (reinterpret_cast<uintptr_t>(sf) & sf_mask) ||
+      (reinterpret_cast<uintptr_t>(sft) & sf_mask))
+    return FP8Q_ERR_ALIGN;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_quantize_rowwise_colwise(dev, x, rows, cols, flags, q, sf, qt, sft, as_stream(stream));
 }
 
 size_t fp8q_permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts) {

@@ -2,6 +2,8 @@
 // Not part of the public ABI; arguments are assumed validated by the caller.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,6 +21,9 @@ struct DeviceInfo {
 // word's device address with the device current.
 fp8q_status device_info(DeviceInfo* out);
 
+// cuTensorMapEncodeTiled from the driver, or nullptr when it cannot be had.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
 // Row-wise quantization of n_tiles consecutive 128-element bf16 tiles:
 // x[n_tiles*128] -> q[n_tiles*128], sf[n_tiles].  With limit_rows (a device int32),
 // only the first limit_rows[0] * tiles_per_row tiles are processed.
@@ -35,6 +40,10 @@ fp8q_status launch_naive_transpose(const DeviceInfo& dev, const uint8_t* q, cons
 
 fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const void* up, int64_t rows, int64_t cols,
                                 uint8_t* q, uint8_t* sf, uint8_t* qt, uint8_t* sft, cudaStream_t stream);
+
+fp8q_status launch_quantize_rowwise_colwise(const DeviceInfo& dev, const void* x, int64_t rows, int64_t cols,
+                                            uint32_t flags, uint8_t* q, void* sf, uint8_t* qt, void* sft,
+                                            cudaStream_t stream);
 
 size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts);
 fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,

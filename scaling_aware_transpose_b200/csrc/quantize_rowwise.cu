@@ -21,37 +21,6 @@ constexpr int kQThreads = 256;
 constexpr int kQUnroll = 2;        // tile slots per thread, all loads issued first
 constexpr int kTilesPerWarp = 4;   // 8 lanes per tile, 16 elements per lane
 
-// Two bf16x2 words -> the larger magnitude per half (sign bits meaningless).
-__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-// Scale exponent of a tile from its BF16 amax bit pattern (sign clear): e = the smallest
-// integer with amax <= 448 * 2^e, 0 for amax == 0, clamped below at -127.  With
-// amax = (1 + m/128) * 2^(E-127): e = E - 135, plus one when the 7-bit mantissa exceeds
-// 0x60 (mu > 1.75 = 448 / 2^8).  BF16 subnormals (E == 0) are all far below the clamp.
-__device__ __forceinline__ int bf16_tile_exponent(uint32_t amax16) {
-  const int e = (int)(amax16 >> 7) - 135 + ((amax16 & 0x7Fu) > 0x60u ? 1 : 0);
-  return amax16 == 0u ? 0 : max(e, -127);
-}
-
-// Four bf16 (two words) times s -> four E4M3 codes, element 0 in the low byte.  The
-// product by a power of two is exact except below 2^-126, where E4M3 rounds to +-0
-// either way.
-__device__ __forceinline__ uint32_t encode4(uint32_t a, uint32_t b, float s) {
-  float2 p0 = make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
-  float2 p1 = make_float2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u));
-  uint64_t r0, r1;
-  const uint64_t ss = ((uint64_t)__float_as_uint(s) << 32) | __float_as_uint(s);
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r0) : "l"(*reinterpret_cast<uint64_t*>(&p0)), "l"(ss));
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r1) : "l"(*reinterpret_cast<uint64_t*>(&p1)), "l"(ss));
-  const uint32_t c01 = cvt_e4m3x2_f32(__uint_as_float((uint32_t)r0), __uint_as_float((uint32_t)(r0 >> 32)));
-  const uint32_t c23 = cvt_e4m3x2_f32(__uint_as_float((uint32_t)r1), __uint_as_float((uint32_t)(r1 >> 32)));
-  return __byte_perm(c01, c23, 0x5410);
-}
-
 // limit_rows (optional, device): only the first limit_rows[0] * tiles_per_row tiles are
 // processed (the valid rows of a grouped buffer, known only on the device).
 // Lane l of a warp serves tile 4*slot + l/8; its 16 elements are 8 from each half of

@@ -96,6 +96,32 @@ def test_swiglu_host_errors(L):
     assert f(None, None, 0, 256, None, None, None, None, None) == sat.FP8Q_OK
 
 
+def test_rowwise_colwise_host_errors(L):
+    f = L.fp8q_quantize_rowwise_colwise
+    Z, P = sat.ZERO_TILE_MIN_SCALE, sat.SF_PACKED_UE8M0
+    assert f(A, 256, 100, 0, A, A, A, A, None) == sat.FP8Q_ERR_SHAPE        # cols % 128
+    assert f(A, 100, 256, 0, A, A, A, A, None) == sat.FP8Q_ERR_SHAPE        # column-wise needs rows % 128
+    assert f(A, 256, 256, 4, A, A, A, A, None) == sat.FP8Q_ERR_ARG          # unknown flag bit
+    assert f(A, 256, 256, 0, A, A, A, None, None) == sat.FP8Q_ERR_ARG       # qt without sft
+    assert f(A, 256, 256, 0, A, A, None, A, None) == sat.FP8Q_ERR_ARG       # sft without qt
+    assert f(None, 256, 256, 0, A, A, None, None, None) == sat.FP8Q_ERR_NULL
+    assert f(A, 256, 256, 0, A, None, A, A, None) == sat.FP8Q_ERR_NULL
+    assert f(MIS, 256, 256, Z, A, A, A, A, None) == sat.FP8Q_ERR_ALIGN
+    assert f(A, 256, 256, 0, A, A, MIS, A, None) == sat.FP8Q_ERR_ALIGN      # qt must be 16-byte aligned
+    assert f(A, 256, 256, P, A, A + 2, A, A, None) == sat.FP8Q_ERR_ALIGN    # packed words: 4-byte aligned
+    assert f(A, 256, 256, P, A, A, A, A + 1, None) == sat.FP8Q_ERR_ALIGN
+    assert f(None, 0, 256, Z | P, None, None, None, None, None) == sat.FP8Q_OK  # empty: no-op
+    assert f(A, 1 << 31, 128, 0, A, A, None, None, None) == sat.FP8Q_ERR_SHAPE
+
+
+def test_packed_sf_bytes(L):
+    assert sat.fp8q_packed_sf_bytes(8192, 7168) == 4 * 14 * 8192
+    assert sat.fp8q_packed_sf_bytes(7168, 8192) == 4 * 16 * 7168
+    assert sat.fp8q_packed_sf_bytes(3, 640) == 4 * 2 * 4      # K tiles 5 -> 2 words; mn 3 -> 4
+    assert sat.fp8q_packed_sf_bytes(0, 128) == 0
+    assert sat.packed_sf_shape(3, 640) == (2, 4)
+
+
 def test_permute_host_errors(L):
     f = L.fp8q_permute_pad_quant
 
