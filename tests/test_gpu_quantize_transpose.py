@@ -43,8 +43,8 @@ def test_tiny_config():
     check_against_oracle(synthetic.tiny()["x"], naive=True)
 
 
-# rows x cols: several tiles, ragged warp shares (tile counts not a multiple of the
-# persistent grid's warps), a single tile, odd column-block counts
+# rows x cols: several tiles, block counts that leave a partial last wave of CTAs, a
+# single tile, odd column-block counts
 SHAPES = [(128, 128), (128, 384), (256, 640), (384, 1152), (640, 256), (1024, 1024), (1152, 896), (2048, 7168)]
 
 
