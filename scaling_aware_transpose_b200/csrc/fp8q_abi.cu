@@ -33,20 +33,6 @@ fp8q_status device_info(DeviceInfo* out) {
   return FP8Q_OK;
 }
 
-// The driver's tensor-map encoder, fetched through the runtime once (no libcuda link).
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // ---- bounded-wait test hook: one mbarrier nobody arrives at
 __global__ void expire_wait_kernel(uint64_t timeout_ns, int* status) {
   __shared__ uint64_t bar;

@@ -2,8 +2,6 @@
 // Not part of the public ABI; arguments are assumed validated by the caller.
 #pragma once
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,9 +18,6 @@ struct DeviceInfo {
 // Per-device facts, queried once per device and cached; also resolves the status
 // word's device address with the device current.
 fp8q_status device_info(DeviceInfo* out);
-
-// cuTensorMapEncodeTiled from the driver, or nullptr when it cannot be had.
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Row-wise quantization of n_tiles consecutive 128-element bf16 tiles:
 // x[n_tiles*128] -> q[n_tiles*128], sf[n_tiles].  With limit_rows (a device int32),
