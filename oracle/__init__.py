@@ -65,6 +65,7 @@ def _declare(L):
         "orc_swiglu_quant": [V, V, I64, I64, V, V, V, V],
         "orc_permute_pad_quant": [V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
         "orc_quantize_rowwise_colwise": [V, I64, I64, ctypes.c_uint32, V, V, V, V],
+        "orc_unpermute_unpad": [V, V, I64, I64, V, V, I64, I32, V],
     }.items():
         fn = getattr(L, name)
         fn.argtypes, fn.restype = args, ctypes.c_int
@@ -263,6 +264,30 @@ def permute_pad_quant(x_bits, topk_idx, num_experts: int, align: int, max_rows: 
     if rc:
         raise OracleError(f"oracle permute_pad_quant rejected its arguments (code {rc})")
     return q, sf, off, rmap
+
+
+def unpermute_unpad(y, row_id_map, topk: int, weights=None, y_sf=None):
+    """Combine side: out bf16 bits [T, H] = sum_s w[t,s] * Y[row_id_map[t,s]] (fp32 fma
+    chain in slot order, BF16 RNE).  y is bf16 bits [rows, H], or E4M3 codes [rows, H]
+    with y_sf [rows, H/128].  row_id_map [T*topk] (or [T, topk]); weights fp32
+    [T, topk] or None (all ones)."""
+    rmap = _c(row_id_map, np.int32).reshape(-1, topk)
+    T, K = rmap.shape
+    if y_sf is None:
+        yy = _c(y, np.uint16)
+        sf = None
+    else:
+        yy = _c(y, np.uint8)
+        sf = _c(y_sf, np.uint8)
+    rows, H = yy.shape
+    w = None if weights is None else _c(weights, np.float32)
+    if w is not None and w.shape != (T, K):
+        raise OracleError("weights must be [tokens, topk]")
+    out = np.empty((T, H), np.uint16)
+    rc = lib().orc_unpermute_unpad(_p(yy), _p(sf), rows, H, _p(rmap), _p(w), T, K, _p(out))
+    if rc:
+        raise OracleError(f"oracle unpermute rejected its arguments (code {rc})")
+    return out
 
 
 def num_threads() -> int:

@@ -669,6 +669,52 @@ int orc_permute_pad_quant(const uint16_t *x, int64_t T, int64_t H, const int32_t
     return 0;
 }
 
+/* ------------------------------------------------------------------ */
+/* Fused unpermute + unpad ([FLOW] 核心方法: Fused Permute+Padding /    */
+/* Unpermute+Unpadding; the combine side of the expert path)           */
+/* ------------------------------------------------------------------ */
+
+/* Expert-ordered rows Y (the permuted, padded buffer after the expert) -> one BF16
+ * row per token: out[t] = sum over slots s of w[t,s] * Y[row_id_map[t,s]].  The
+ * padding rows are simply never read (unpad).  With w == NULL every weight is 1: the
+ * backward of the permute, which sums the gradients of a token's K copies.
+ * Y is either BF16 (y_sf == NULL) or row-wise FP8: E4M3 codes with UE8M0 scales
+ * [rows, H/128], dequantized to fp32 as decode(q) * 2^e (exact unless the product
+ * overflows fp32, which only codes >= 256 at e >= 120 can).
+ * Reading (the pages fix no arithmetic for the combine): accumulate in fp32, one
+ * fused multiply-add per slot in slot order s = 0..K-1 starting from +0, then round
+ * to BF16 with round-to-nearest-even.  Results must be finite (NaN unspecified).
+ * Returns 0, 2 (shape), 7 (a row index outside [0, rows)). */
+int orc_unpermute_unpad(const void *y, const uint8_t *y_sf, int64_t rows, int64_t H, const int32_t *row_id_map,
+                        const float *w, int64_t T, int32_t K, uint16_t *out)
+{
+    if (H % 128 || T < 0 || K < 1 || rows < 0)
+        return 2;
+    for (int64_t p = 0; p < T * K; p++)
+        if (row_id_map[p] < 0 || row_id_map[p] >= rows)
+            return 7;
+    int64_t nt = H / 128;
+    const uint16_t *yb = (const uint16_t *)y;
+    const uint8_t *yq = (const uint8_t *)y;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; t++)
+        for (int64_t h = 0; h < H; h++) {
+            float acc = 0.0f;
+            for (int32_t s = 0; s < K; s++) {
+                int64_t r = row_id_map[t * K + s];
+                float v;
+                if (y_sf)
+                    v = (float)ldexp(orc_e4m3_decode(yq[r * H + h]), (int)y_sf[r * nt + h / 128] - 127);
+                else
+                    v = (float)bf16_to_double(yb[r * H + h]);
+                float ws = w ? w[t * K + s] : 1.0f;
+                acc = fmaf(ws, v, acc);
+            }
+            out[t * H + h] = f32_to_bf16_rne(acc);
+        }
+    return 0;
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

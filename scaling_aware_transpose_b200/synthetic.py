@@ -81,6 +81,18 @@ def moe(seed: int = 0, tokens: int = 16384, hidden: int = 7168, num_experts: int
     return {"x": _bf16_bits(x), "topk_idx": idx, "num_experts": num_experts}
 
 
+def moe_combine(seed: int = 0, tokens: int = 16384, hidden: int = 7168, rows: int = 133120,
+                topk: int = 8) -> dict:
+    """Combine-side inputs of the MoE workload: expert outputs Y bf16 [rows, hidden] ~
+    N(0,1) (the permuted, padded buffer after the expert GEMMs) and routing weights
+    fp32 [tokens, topk] drawn from a flat Dirichlet (positive, each token's weights sum
+    to 1, like normalised router probabilities)."""
+    rng = np.random.default_rng(seed + 1000)
+    y = rng.standard_normal((rows, hidden), dtype=np.float32)
+    w = rng.dirichlet(np.ones(topk), size=tokens).astype(np.float32)
+    return {"y": _bf16_bits(y), "weights": np.ascontiguousarray(w)}
+
+
 def swiglu(seed: int = 0, rows: int = 32768, cols: int = 2048) -> dict:
     """gate, up bf16 [32768, 2048], independent N(0,1), both multiplied by one
     lognormal(0, 1) factor per row (reading: "N(0,1) times per-row lognormal(0,1)"

@@ -52,3 +52,13 @@ def test_zipf_topk_distinct_and_skewed():
     counts = np.bincount(idx.ravel(), minlength=32)
     assert counts[0] > counts[15] > counts[31]
     assert counts.sum() == 4096 * 8
+
+
+def test_moe_combine_inputs():
+    d = synthetic.moe_combine(tokens=300, hidden=256, rows=2500, topk=8, seed=2)
+    assert d["y"].shape == (2500, 256) and d["y"].dtype == np.uint16
+    w = d["weights"]
+    assert w.shape == (300, 8) and w.dtype == np.float32 and np.all(w > 0)
+    assert np.allclose(w.astype(np.float64).sum(axis=1), 1.0, atol=1e-6)
+    again = synthetic.moe_combine(tokens=300, hidden=256, rows=2500, topk=8, seed=2)
+    assert np.array_equal(again["y"], d["y"]) and np.array_equal(again["weights"], w)
