@@ -682,8 +682,10 @@ int orc_permute_pad_quant(const uint16_t *x, int64_t T, int64_t H, const int32_t
  * [rows, H/128], dequantized to fp32 as decode(q) * 2^e (exact unless the product
  * overflows fp32, which only codes >= 256 at e >= 120 can).
  * Reading (the pages fix no arithmetic for the combine): accumulate in fp32, one
- * fused multiply-add per slot in slot order s = 0..K-1 starting from +0, then round
- * to BF16 with round-to-nearest-even.  Results must be finite (NaN unspecified).
+ * fused multiply-add per slot in slot order s = 0..K-1 starting from -0 (the additive
+ * identity that also keeps the sign of a zero product, so one slot gives its product
+ * exactly and K = 1 inverts the permute bit for bit), then round to BF16 with
+ * round-to-nearest-even.  Results must be finite (NaN unspecified).
  * Returns 0, 2 (shape), 7 (a row index outside [0, rows)). */
 int orc_unpermute_unpad(const void *y, const uint8_t *y_sf, int64_t rows, int64_t H, const int32_t *row_id_map,
                         const float *w, int64_t T, int32_t K, uint16_t *out)
@@ -699,7 +701,7 @@ int orc_unpermute_unpad(const void *y, const uint8_t *y_sf, int64_t rows, int64_
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; t++)
         for (int64_t h = 0; h < H; h++) {
-            float acc = 0.0f;
+            float acc = -0.0f;
             for (int32_t s = 0; s < K; s++) {
                 int64_t r = row_id_map[t * K + s];
                 float v;

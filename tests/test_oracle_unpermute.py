@@ -54,14 +54,14 @@ def test_golden_examples():
             out = oracle.unpermute_unpad(y, np.array(rows, np.int32), 2, wts, y_sf=sf)
             assert np.all(out == want), (name, hex(int(out[0, 0])), hex(want))
             n += 1
-    assert n == 9
+    assert n == 12
 
 
 def emulate(y_f32, rmap, w):
     """The same fp32 fma chain, emulated in float64 (a*b is exact in double; the sum is
     rounded once to double, then to float32), BF16 rounding by torch."""
     T, K = rmap.shape
-    acc = np.zeros((T, y_f32.shape[1]), np.float32)
+    acc = np.full((T, y_f32.shape[1]), -0.0, np.float32)
     for s in range(K):
         ws = np.ones(T, np.float64) if w is None else w[:, s].astype(np.float64)
         acc = (ws[:, None] * y_f32[rmap[:, s]].astype(np.float64) + acc.astype(np.float64)).astype(np.float32)
@@ -103,10 +103,12 @@ def test_permute_round_trip_bf16():
     assert np.array_equal(oracle.unpermute_unpad(y, rmap, 1), d["x"])
 
 
-def test_permute_round_trip_fp8():
+@pytest.mark.parametrize("seed", [5, 8])
+def test_permute_round_trip_fp8(seed):
     """K = 1 on the FP8 permute output: the BF16 rounding of the row-wise dequantization
-    (torch decodes the codes) - the permute's rows come back to their tokens."""
-    d = synthetic.moe(tokens=150, hidden=384, num_experts=5, topk=1, seed=5)
+    (torch decodes the codes) - the permute's rows come back to their tokens, codes of
+    -0 included."""
+    d = synthetic.moe(tokens=150 * seed, hidden=384, num_experts=5, topk=1, seed=seed)
     pq, psf, off, rmap = oracle.permute_pad_quant(d["x"], d["topk_idx"], 5, 128)
     q, sf = oracle.quantize_rowwise(d["x"])
     dec = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float64).numpy()
