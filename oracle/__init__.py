@@ -66,6 +66,7 @@ def _declare(L):
         "orc_permute_pad_quant": [V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
         "orc_quantize_rowwise_colwise": [V, I64, I64, ctypes.c_uint32, V, V, V, V],
         "orc_unpermute_unpad": [V, V, I64, I64, V, V, I64, I32, V],
+        "orc_permute_pad_fp8": [V, V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
     }.items():
         fn = getattr(L, name)
         fn.argtypes, fn.restype = args, ctypes.c_int
@@ -264,6 +265,28 @@ def permute_pad_quant(x_bits, topk_idx, num_experts: int, align: int, max_rows: 
     if rc:
         raise OracleError(f"oracle permute_pad_quant rejected its arguments (code {rc})")
     return q, sf, off, rmap
+
+
+def permute_pad_fp8(q_bits, sf, topk_idx, num_experts: int, align: int, max_rows: int | None = None,
+                    fill: int = 0xEE):
+    """FP8-input permute + pad: the same outputs as permute_pad_quant, from row-wise codes
+    q [T, H] and scales sf [T, H/128] instead of BF16 X."""
+    xq = _c(q_bits, np.uint8)
+    xsf = _c(sf, np.uint8)
+    idx = _c(topk_idx, np.int32)
+    T, H = xq.shape
+    K = idx.shape[1] if idx.ndim == 2 else 1
+    if max_rows is None:
+        max_rows = permute_max_rows(T, K, num_experts, align)
+    q = np.full((max_rows, H), fill, np.uint8)
+    osf = np.full((max_rows, H // 128), fill, np.uint8)
+    off = np.zeros(num_experts + 1, np.int32)
+    rmap = np.zeros(T * K, np.int32)
+    rc = lib().orc_permute_pad_fp8(_p(xq), _p(xsf), T, H, _p(idx), K, num_experts, align, _p(q), _p(osf), max_rows,
+                                   _p(off), _p(rmap))
+    if rc:
+        raise OracleError(f"oracle FP8 permute rejected its arguments (code {rc})")
+    return q, osf, off, rmap
 
 
 def unpermute_unpad(y, row_id_map, topk: int, weights=None, y_sf=None):

@@ -669,6 +669,60 @@ int orc_permute_pad_quant(const uint16_t *x, int64_t T, int64_t H, const int32_t
     return 0;
 }
 
+/* FP8-input permute + pad ([FLOW] 核心方法 with the pages' FP8 dataflow: the
+ * dispatch already delivers row-wise FP8 codes and their scales, so the permute moves
+ * codes instead of quantizing).  Same routing, offsets, padding and return codes as
+ * orc_permute_pad_quant; the payload of row (t, s) is the token's codes and scale
+ * bytes, copied. */
+int orc_permute_pad_fp8(const uint8_t *xq, const uint8_t *xsf, int64_t T, int64_t H, const int32_t *idx, int32_t K,
+                        int32_t E, int32_t align, uint8_t *q, uint8_t *sf, int64_t max_rows, int32_t *offsets,
+                        int32_t *row_id_map)
+{
+    if (H % 128 || T < 0 || K < 1 || E < 1 || align < 1)
+        return 2;
+    int64_t nt = H / 128;
+    int64_t *cnt = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    if (!cnt)
+        return 5;
+    for (int64_t p = 0; p < T * K; p++) {
+        if (idx[p] < 0 || idx[p] >= E) {
+            free(cnt);
+            return 7;
+        }
+        cnt[idx[p]]++;
+    }
+    int64_t acc = 0;
+    for (int32_t e = 0; e < E; e++) {
+        offsets[e] = (int32_t)acc;
+        acc += (cnt[e] + align - 1) / align * align;
+    }
+    offsets[E] = (int32_t)acc;
+    if (acc > max_rows) {
+        free(cnt);
+        return 4;
+    }
+    int64_t *seen = cnt;
+    memset(seen, 0, (size_t)E * sizeof(int64_t));
+    for (int64_t p = 0; p < T * K; p++) {
+        int32_t e = idx[p];
+        row_id_map[p] = (int32_t)(offsets[e] + seen[e]);
+        seen[e]++;
+    }
+    for (int64_t t = 0; t < T; t++)
+        for (int32_t s = 0; s < K; s++) {
+            int64_t r = row_id_map[t * K + s];
+            memcpy(q + r * H, xq + t * H, (size_t)H);
+            memcpy(sf + r * nt, xsf + t * nt, (size_t)nt);
+        }
+    for (int32_t e = 0; e < E; e++)
+        for (int64_t r = offsets[e] + seen[e]; r < offsets[e + 1]; r++) {
+            memset(q + r * H, 0x00, (size_t)H);
+            memset(sf + r * nt, 127, (size_t)nt);
+        }
+    free(cnt);
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* Fused unpermute + unpad ([FLOW] 核心方法: Fused Permute+Padding /    */
 /* Unpermute+Unpadding; the combine side of the expert path)           */

@@ -151,3 +151,42 @@ def test_permute_rejects_bad_index():
     x = synthetic.scaled_normal(4, 128, seed=14)
     with pytest.raises(oracle.OracleError):
         oracle.permute_pad_quant(x, np.array([[0], [1], [5], [2]], np.int32), 4, 16)
+
+
+# ------------------------------------------------------------------ FP8-input permute
+
+@pytest.mark.parametrize("T,H,K,E,align", [(64, 256, 2, 4, 16), (300, 384, 8, 32, 128), (1, 128, 1, 1, 1),
+                                           (129, 128, 3, 5, 7)])
+def test_fp8_permute_equals_quantize_then_permute(T, H, K, E, align):
+    """Quantization is row-local, so permuting the row-wise codes and scales must give
+    byte for byte what the fused BF16 permute+quantize gives (same routing, offsets,
+    padding rows)."""
+    d = synthetic.moe(tokens=T, hidden=H, num_experts=E, topk=K, seed=T + E)
+    q, sf = oracle.quantize_rowwise(d["x"])
+    a = oracle.permute_pad_fp8(q, sf, d["topk_idx"], E, align)
+    b = oracle.permute_pad_quant(d["x"], d["topk_idx"], E, align)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_fp8_permute_brute_force_rows():
+    """Pure-Python gather: row row_id_map[t*K+s] holds token t's codes and scales."""
+    d = synthetic.moe(tokens=40, hidden=256, num_experts=3, topk=2, seed=1)
+    rng = np.random.default_rng(0)
+    q = rng.integers(0, 256, size=(40, 256), dtype=np.uint8)
+    sf = rng.integers(100, 140, size=(40, 2), dtype=np.uint8)
+    oq, osf, off, rmap = oracle.permute_pad_fp8(q, sf, d["topk_idx"], 3, 16)
+    for p in range(80):
+        t = p // 2
+        assert np.array_equal(oq[rmap[p]], q[t]) and np.array_equal(osf[rmap[p]], sf[t])
+    used = set(rmap.tolist())
+    for r in range(int(off[-1])):
+        if r not in used:
+            assert np.all(oq[r] == 0) and np.all(osf[r] == 127)
+
+
+def test_fp8_permute_bad_index():
+    q = np.zeros((4, 128), np.uint8)
+    sf = np.full((4, 1), 127, np.uint8)
+    with pytest.raises(oracle.OracleError):
+        oracle.permute_pad_fp8(q, sf, np.array([[0], [1], [9], [2]], np.int32), 4, 16)
