@@ -190,8 +190,9 @@ def measure_workloads(reps, device, stream, flush, peak):
     """The other hot-path rows on their own workloads, each kernel after an L2 flush:
     fused SwiGLU+quantize(+transpose) on gate/up [32768, 2048]; fused permute+pad(128)+
     quantize of X [16384, 7168] with top-8 of 32 Zipf(1.1) experts, then the grouped
-    direct transpose on its device offsets; quantize + direct transpose on the range-
-    stress X [65536, 7168]."""
+    direct transpose on its device offsets, and the combine-side unpermute+unpad of BF16
+    expert outputs (weighted) and of the FP8 rows (unit weights); quantize + direct
+    transpose on the range-stress X [65536, 7168]."""
     import torch
 
     import scaling_aware_transpose_b200 as sat
@@ -237,14 +238,40 @@ def measure_workloads(reps, device, stream, flush, peak):
                                               ws.numel(), sp)
     t_perm = time_on_stream(perm, reps + 2, stream, lambda: flush.fill_(6))
     R = int(off[-1].item())
+    # FP8-input permute (the dispatch delivered row-wise codes and scales): same routing,
+    # rows copied instead of quantized
+    xq, xsf = sat.quantize_rowwise(x)
+    q8 = torch.empty_like(q)
+    sf8 = torch.empty_like(sf)
+    perm8 = lambda: sat.fp8q_permute_pad_fp8(xq, xsf, T, H, idx, K, E, align, q8, sf8, max_rows, off, rmap, ws,
+                                             ws.numel(), sp)
+    t_perm8 = time_on_stream(perm8, reps + 2, stream, lambda: flush.fill_(14))
+    del xq, xsf, q8, sf8
     qt = torch.empty(max_rows * H, dtype=torch.uint8, device=device)
     sft = torch.empty(max_rows * H // 128, dtype=torch.uint8, device=device)
     t_gt = time_on_stream(lambda: sat.fp8q_direct_transpose(q, sf, max_rows, H, off, E, qt, sft, sp), reps + 2,
                           stream, lambda: flush.fill_(7))
     perm_bytes = 2 * T * H + 4 * T * K + R * (H + H // 128) + 4 * (E + 1) + 4 * T * K
     out[f"permute_pad_quant [16384x7168] top8/32 -> {R} rows"] = entry(perm_bytes, t_perm)
+    perm8_bytes = T * (H + H // 128) + 4 * T * K + R * (H + H // 128) + 4 * (E + 1) + 4 * T * K
+    out[f"permute_pad_fp8 [16384x7168] top8/32 -> {R} rows"] = entry(perm8_bytes, t_perm8)
     out[f"direct_transpose grouped [{R}x7168] 32 experts"] = entry(2 * R * (H + H // 128), t_gt)
-    del x, idx, q, sf, off, rmap, ws, qt, sft
+    del qt, sft
+    # combine side: unpermute + unpad of BF16 expert outputs with routing weights, and of
+    # the FP8 rows with unit weights (the permute's backward shape)
+    c = synthetic.moe_combine(rows=R, topk=K)
+    y = synthetic.to_torch_bf16(c["y"]).to(device)
+    wts = torch.from_numpy(c["weights"]).to(device)
+    comb = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    t_ub = time_on_stream(lambda: sat.fp8q_unpermute_unpad(y, None, R, H, rmap, wts, T, K, comb, sp), reps + 2,
+                          stream, lambda: flush.fill_(12))
+    t_uq = time_on_stream(lambda: sat.fp8q_unpermute_unpad(q, sf, max_rows, H, rmap, None, T, K, comb, sp), reps + 2,
+                          stream, lambda: flush.fill_(13))
+    out[f"unpermute_unpad bf16 [{R}x7168] -> [16384x7168], weighted"] = entry(
+        T * K * 2 * H + 2 * T * H + 8 * T * K, t_ub)
+    out[f"unpermute_unpad fp8 [{R}x7168] -> [16384x7168], unit weights"] = entry(
+        T * K * (H + H // 128) + 2 * T * H + 4 * T * K, t_uq)
+    del x, idx, q, sf, off, rmap, ws, y, wts, comb
     # range stress
     d = synthetic.stress()
     x = synthetic.to_torch_bf16(d["x"]).to(device)
@@ -529,6 +556,17 @@ def run_profile(args):
         qt = torch.empty((C, R), dtype=torch.uint8, device="cuda")
         sft = torch.empty((C, R // 128), dtype=torch.uint8, device="cuda")
         calls = {"swiglu": lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, qt, sft)}
+    elif args.profile == "unpermute":
+        d = synthetic.moe()
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        K = idx.shape[1]
+        pq, psf, off, rmap = sat.permute_pad_quant(x, idx, d["num_experts"], 128)
+        R = int(off[-1].item())
+        c = synthetic.moe_combine(rows=R, topk=K)
+        y = synthetic.to_torch_bf16(c["y"]).cuda()
+        wts = torch.from_numpy(c["weights"]).cuda()
+        calls = {"unpermute": lambda: sat.unpermute_unpad(y, rmap, K, wts)}
     else:  # permute
         d = synthetic.moe()
         x = synthetic.to_torch_bf16(d["x"]).cuda()
@@ -553,7 +591,8 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true", help="skip the SwiGLU / MoE / stress workload timings")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
-    ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise"],
+    ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise",
+                                          "unpermute"],
                     default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)

@@ -190,6 +190,46 @@ fp8q_status fp8q_quantize_rowwise_colwise(const void *x, int64_t rows, int64_t c
                                           uint8_t *q, void *sf, uint8_t *qt, void *sft,
                                           fp8q_stream_t stream);
 
+/* Fused unpermute + unpad: the combine side of the expert path (FP8-Flow-MoE 核心方法,
+ * fused Unpermute+Unpadding).  Each token gathers its K expert rows back and sums them
+ * with its routing weights; padding rows are never read:
+ *   out[t, h] = BF16_RNE( fma chain over s = 0..K-1 of w[t,s] * v(row_id_map[t,s], h) ),
+ * acc starting at -0 (so one slot gives its product exactly, sign of zero included),
+ * one fp32 fused multiply-add per slot in slot order, where v is the fp32 value of the
+ * row element (this order is the library's reading; the pages fix none).
+ *   y          : BF16 [rows, hidden] when y_sf is NULL, else E4M3 codes u8 [rows, hidden]
+ *                with y_sf u8 [rows, hidden/128] row-wise UE8M0 scales (v = decode(q) *
+ *                2^(byte - 127), exact unless it overflows fp32).  hidden % 128 == 0.
+ *   rows       : rows of y (the permuted buffer's capacity).
+ *   row_id_map : int32 [tokens, topk], as written by fp8q_permute_pad_quant.  An entry
+ *                outside [0, rows) sets FP8Q_ERR_DEVICE in the status word and its slot
+ *                is skipped.
+ *   weights    : fp32 [tokens, topk] routing weights, or NULL for all ones (the
+ *                backward of the permute: the sum of a token's K row gradients).
+ *   out        : BF16 [tokens, hidden].
+ * Results must be finite (NaN outputs are unspecified).  y and out 16-byte aligned;
+ * row_id_map and weights 4-byte aligned.  Errors: NULL, ALIGN, SHAPE, ARG (topk not in
+ * [1, 64]), CUDA. */
+fp8q_status fp8q_unpermute_unpad(const void *y, const uint8_t *y_sf, int64_t rows, int64_t hidden,
+                                 const int32_t *row_id_map, const float *weights, int64_t tokens,
+                                 int32_t topk, void *out, fp8q_stream_t stream);
+
+/* FP8-input permute + pad: the pages' FP8 dataflow quantizes before the dispatch, so the
+ * permute receives row-wise codes and scales (FP8-Flow-MoE 核心方法 and casting-free
+ * dataflow).  Same routing, offsets, row ids, padding rows and errors as
+ * fp8q_permute_pad_quant; the payload of a destination row is the token's codes and
+ * scale bytes, copied:
+ *   xq  : u8 [tokens, hidden] E4M3 codes, 16-byte aligned;
+ *   xsf : u8 [tokens, hidden/128] UE8M0 scale bytes.
+ * All other arguments and the workspace (fp8q_permute_workspace_bytes) as in
+ * fp8q_permute_pad_quant.  Permuting quantize_rowwise(X) this way gives byte for byte
+ * what fp8q_permute_pad_quant(X) gives. */
+fp8q_status fp8q_permute_pad_fp8(const uint8_t *xq, const uint8_t *xsf, int64_t tokens, int64_t hidden,
+                                 const int32_t *topk_idx, int32_t topk, int32_t num_experts, int32_t align,
+                                 uint8_t *q, uint8_t *sf, int64_t max_out_rows, int32_t *expert_offsets,
+                                 int32_t *row_id_map, void *workspace, size_t workspace_bytes,
+                                 fp8q_stream_t stream);
+
 /* Size of the library's static scratch for fp8q_permute_pad_quant_noalloc (4 MiB). */
 #define FP8Q_NOALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -56,7 +56,9 @@ def lib() -> ctypes.CDLL:
             "fp8q_quantize_rowwise_colwise": ([P, I64, I64, ctypes.c_uint32, P, P, P, P, P], ctypes.c_int),
             "fp8q_permute_workspace_bytes": ([I64, I32, I32], SZ),
             "fp8q_permute_pad_quant": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
+            "fp8q_permute_pad_fp8": ([P, P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
             "fp8q_permute_pad_quant_noalloc": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P], ctypes.c_int),
+            "fp8q_unpermute_unpad": ([P, P, I64, I64, P, P, I64, I32, P, P], ctypes.c_int),
             "fp8q_debug_expire_wait": ([ctypes.c_uint64, P], ctypes.c_int),
             "fp8q_version": ([], ctypes.c_int),
         }
@@ -151,6 +153,14 @@ def fp8q_permute_workspace_bytes(tokens: int, topk: int, num_experts: int) -> in
     return int(lib().fp8q_permute_workspace_bytes(tokens, topk, num_experts))
 
 
+def fp8q_permute_pad_fp8(xq, xsf, tokens: int, hidden: int, topk_idx, topk: int, num_experts: int, align: int,
+                         q, sf, max_out_rows: int, expert_offsets, row_id_map, workspace, workspace_bytes: int,
+                         stream=None) -> None:
+    _check(lib().fp8q_permute_pad_fp8(_ptr(xq), _ptr(xsf), tokens, hidden, _ptr(topk_idx), topk, num_experts, align,
+                                      _ptr(q), _ptr(sf), max_out_rows, _ptr(expert_offsets), _ptr(row_id_map),
+                                      _ptr(workspace), workspace_bytes, _stream(stream)), "fp8q_permute_pad_fp8")
+
+
 def fp8q_permute_pad_quant(x, tokens: int, hidden: int, topk_idx, topk: int, num_experts: int, align: int,
                            q, sf, max_out_rows: int, expert_offsets, row_id_map, workspace,
                            workspace_bytes: int, stream=None) -> None:
@@ -172,6 +182,12 @@ def fp8q_permute_pad_quant_noalloc(x, tokens: int, hidden: int, topk_idx, topk: 
                                                 align, _ptr(q), _ptr(sf), max_out_rows, _ptr(expert_offsets),
                                                 _ptr(row_id_map), _stream(stream)),
            "fp8q_permute_pad_quant_noalloc")
+
+
+def fp8q_unpermute_unpad(y, y_sf, rows: int, hidden: int, row_id_map, weights, tokens: int, topk: int, out,
+                         stream=None) -> None:
+    _check(lib().fp8q_unpermute_unpad(_ptr(y), _ptr(y_sf), rows, hidden, _ptr(row_id_map), _ptr(weights), tokens,
+                                      topk, _ptr(out), _stream(stream)), "fp8q_unpermute_unpad")
 
 
 def fp8q_debug_expire_wait(timeout_ns: int, stream=None) -> None:
@@ -286,3 +302,34 @@ def permute_pad_quant(x, topk_idx, num_experts: int, align: int, max_out_rows: i
     fp8q_permute_pad_quant(x, tokens, hidden, topk_idx, topk, num_experts, align, q, sf, max_out_rows, off,
                            rmap, ws, ws.numel(), stream)
     return q, sf, off, rmap
+
+
+def permute_pad_fp8(xq, xsf, topk_idx, num_experts: int, align: int, max_out_rows: int | None = None, stream=None):
+    """FP8-input permute: same outputs as permute_pad_quant, from row-wise codes xq
+    [T, H] and scale bytes xsf [T, H/128]."""
+    import torch
+    tokens, hidden = xq.shape
+    topk = topk_idx.shape[1]
+    if max_out_rows is None:
+        max_out_rows = permute_max_rows(tokens, topk, num_experts, align)
+    q = _empty((max_out_rows, hidden), torch.uint8, xq)
+    sf = _empty((max_out_rows, hidden // 128), torch.uint8, xq)
+    off = _empty((num_experts + 1,), torch.int32, xq)
+    rmap = _empty((tokens * topk,), torch.int32, xq)
+    ws_bytes = fp8q_permute_workspace_bytes(tokens, topk, num_experts)
+    ws = _empty((max(ws_bytes, 16),), torch.uint8, xq)
+    fp8q_permute_pad_fp8(xq, xsf, tokens, hidden, topk_idx, topk, num_experts, align, q, sf, max_out_rows, off, rmap,
+                         ws, ws.numel(), stream)
+    return q, sf, off, rmap
+
+
+def unpermute_unpad(y, row_id_map, topk: int, weights=None, y_sf=None, stream=None):
+    """Combine side of the permute: BF16 [tokens, hidden] from the expert-ordered rows y
+    (BF16, or E4M3 codes with row-wise scales y_sf) gathered by row_id_map [tokens*topk]
+    and summed with weights [tokens, topk] (None: all ones)."""
+    import torch
+    rows, hidden = y.shape
+    tokens = row_id_map.numel() // topk
+    out = _empty((tokens, hidden), torch.bfloat16, y)
+    fp8q_unpermute_unpad(y, y_sf, rows, hidden, row_id_map, weights, tokens, topk, out, stream)
+    return out

@@ -68,6 +68,32 @@ fp8q_status check_transpose_args(const uint8_t* q, const uint8_t* sf, int64_t ro
   return FP8Q_OK;
 }
 
+// Rules shared by the two permutes (BF16 input x, or FP8 input x = codes with scales xsf).
+fp8q_status check_permute_args(const void* x, const uint8_t* xsf, bool fp8_input, int64_t tokens, int64_t hidden,
+                               const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
+                               const uint8_t* q, const uint8_t* sf, int64_t max_out_rows,
+                               const int32_t* expert_offsets, const int32_t* row_id_map, const void* workspace,
+                               size_t workspace_bytes) {
+  if (tokens < 0 || hidden < 0 || hidden % 128 || hidden > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (topk < 1 || topk > 64 || num_experts < 1 || num_experts > 4096 || align < 1 || align > 4096) return FP8Q_ERR_ARG;
+  const int64_t need = tokens * topk + (int64_t)num_experts * (align - 1);
+  if (max_out_rows < need || max_out_rows > kMaxDim) return FP8Q_ERR_ARG;
+  if (!expert_offsets) return FP8Q_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(expert_offsets) & 3u)) return FP8Q_ERR_ALIGN;
+  if (tokens > 0) {
+    if (!topk_idx || !row_id_map || !workspace) return FP8Q_ERR_NULL;
+    if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(topk_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(row_id_map) & 3u))
+      return FP8Q_ERR_ALIGN;
+    if (workspace_bytes < fp8q_permute_workspace_bytes(tokens, topk, num_experts)) return FP8Q_ERR_ARG;
+    if (hidden > 0) {
+      if (!x || !q || !sf || (fp8_input && !xsf)) return FP8Q_ERR_NULL;
+      if (!aligned16(x) || !aligned16(q)) return FP8Q_ERR_ALIGN;
+    }
+  }
+  return FP8Q_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -185,27 +211,42 @@ fp8q_status fp8q_permute_pad_quant(const void* x, int64_t tokens, int64_t hidden
                                    int32_t topk, int32_t num_experts, int32_t align, uint8_t* q, uint8_t* sf,
                                    int64_t max_out_rows, int32_t* expert_offsets, int32_t* row_id_map,
                                    void* workspace, size_t workspace_bytes, fp8q_stream_t stream) {
-  if (tokens < 0 || hidden < 0 || hidden % 128 || hidden > kMaxDim) return FP8Q_ERR_SHAPE;
-  if (topk < 1 || topk > 64 || num_experts < 1 || num_experts > 4096 || align < 1 || align > 4096) return FP8Q_ERR_ARG;
-  const int64_t need = tokens * topk + (int64_t)num_experts * (align - 1);
-  if (max_out_rows < need || max_out_rows > kMaxDim) return FP8Q_ERR_ARG;
-  if (!expert_offsets) return FP8Q_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(expert_offsets) & 3u)) return FP8Q_ERR_ALIGN;
-  if (tokens > 0) {
-    if (!topk_idx || !row_id_map || !workspace) return FP8Q_ERR_NULL;
-    if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(topk_idx) & 3u) ||
-        (reinterpret_cast<uintptr_t>(row_id_map) & 3u))
-      return FP8Q_ERR_ALIGN;
-    if (workspace_bytes < fp8q_permute_workspace_bytes(tokens, topk, num_experts)) return FP8Q_ERR_ARG;
-    if (hidden > 0) {
-      if (!x || !q || !sf) return FP8Q_ERR_NULL;
-      if (!aligned16(x) || !aligned16(q)) return FP8Q_ERR_ALIGN;
-    }
-  }
+  const fp8q_status c = check_permute_args(x, nullptr, false, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
+                                           max_out_rows, expert_offsets, row_id_map, workspace, workspace_bytes);
+  if (c != FP8Q_OK) return c;
   fp8q::DeviceInfo dev;
   if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
   return fp8q::launch_permute_pad_quant(dev, x, tokens, hidden, topk_idx, topk, num_experts, align, q, sf, max_out_rows,
                                         expert_offsets, row_id_map, workspace, as_stream(stream));
+}
+
+fp8q_status fp8q_permute_pad_fp8(const uint8_t* xq, const uint8_t* xsf, int64_t tokens, int64_t hidden,
+                                 const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align, uint8_t* q,
+                                 uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets, int32_t* row_id_map,
+                                 void* workspace, size_t workspace_bytes, fp8q_stream_t stream) {
+  const fp8q_status c = check_permute_args(xq, xsf, true, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
+                                           max_out_rows, expert_offsets, row_id_map, workspace, workspace_bytes);
+  if (c != FP8Q_OK) return c;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_permute_pad_fp8(dev, xq, xsf, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
+                                      max_out_rows, expert_offsets, row_id_map, workspace, as_stream(stream));
+}
+
+fp8q_status fp8q_unpermute_unpad(const void* y, const uint8_t* y_sf, int64_t rows, int64_t hidden,
+                                 const int32_t* row_id_map, const float* weights, int64_t tokens, int32_t topk,
+                                 void* out, fp8q_stream_t stream) {
+  if (rows < 0 || hidden < 0 || tokens < 0 || hidden % 128 || rows > kMaxDim || hidden > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (topk < 1 || topk > 64) return FP8Q_ERR_ARG;
+  if (tokens == 0 || hidden == 0) return FP8Q_OK;
+  if (!y || !row_id_map || !out) return FP8Q_ERR_NULL;
+  if (!aligned16(y) || !aligned16(out) || (reinterpret_cast<uintptr_t>(row_id_map) & 3u) ||
+      (reinterpret_cast<uintptr_t>(weights) & 3u))
+    return FP8Q_ERR_ALIGN;
+  fp8q::DeviceInfo dev;
+  if (fp8q::device_info(&dev) != FP8Q_OK) return FP8Q_ERR_CUDA;
+  return fp8q::launch_unpermute_unpad(dev, y, y_sf, rows, hidden, row_id_map, weights, tokens, topk, out,
+                                      as_stream(stream));
 }
 
 fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream) {

@@ -46,6 +46,16 @@ fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64
                                      uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,
                                      int32_t* row_id_map, void* workspace, cudaStream_t stream);
 
+fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const uint8_t* y_sf, int64_t rows,
+                                   int64_t hidden, const int32_t* row_id_map, const float* weights, int64_t tokens,
+                                   int32_t topk, void* out, cudaStream_t stream);
+
+fp8q_status launch_permute_pad_fp8(const DeviceInfo& dev, const uint8_t* xq, const uint8_t* xsf, int64_t tokens,
+                                   int64_t hidden, const int32_t* topk_idx, int32_t topk, int32_t num_experts,
+                                   int32_t align, uint8_t* q, uint8_t* sf, int64_t max_out_rows,
+                                   int32_t* expert_offsets, int32_t* row_id_map, void* workspace,
+                                   cudaStream_t stream);
+
 fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace fp8q

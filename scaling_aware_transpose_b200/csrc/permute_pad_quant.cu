@@ -12,6 +12,8 @@
 // offsets and per-chunk bases, (3) one warp per chunk assigns stable ranks with
 // __match_any_sync, (4) the streaming scatter-quantize over all (token, tile) pairs,
 // (5) zero-fill of the padding rows.  Workspace: counts[C][E], bases[C][E], totals[E].
+// The FP8-input variant (the dispatch already delivered row-wise codes and scales) shares
+// (1)-(3) and (5); its step (4) copies each token's codes and scale bytes to its rows.
 #include "common.cuh"
 #include "launch.h"
 
@@ -204,6 +206,45 @@ __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* _
   }
 }
 
+// FP8-input payload: tiles (token t, column block j) in row-major order, 8 lanes per
+// tile (16 codes each, so each load instruction reads whole 128-byte lines), four tiles
+// per warp per slot, all loads issued first; each tile's codes and scale byte are
+// written to the token's top-k destination rows.
+__global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __restrict__ xq,
+                                                                 const uint8_t* __restrict__ xsf, int64_t tokens,
+                                                                 int ncb, const int32_t* __restrict__ row_id_map,
+                                                                 int topk, uint4* __restrict__ q,
+                                                                 uint8_t* __restrict__ sf) {
+  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int64_t n_tiles = tokens * ncb;
+  const int64_t warp = ((int64_t)blockIdx.x * kSThreads + threadIdx.x) >> 5;
+  int64_t tile[kSUnroll];
+  uint4 v[kSUnroll];
+  uint8_t e[kSUnroll];
+#pragma unroll
+  for (int u = 0; u < kSUnroll; ++u) {
+    tile[u] = (warp * kSUnroll + u) * 4 + (lane >> 3);
+    v[u] = make_uint4(0u, 0u, 0u, 0u);
+    e[u] = 0;
+    if (tile[u] < n_tiles) {
+      v[u] = ld_stream(xq + tile[u] * 8 + sub);
+      if (sub == 0) e[u] = __ldg(xsf + tile[u]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kSUnroll; ++u) {
+    if (tile[u] >= n_tiles) continue;
+    const int64_t t = tile[u] / ncb;
+    const int j = (int)(tile[u] - t * ncb);
+    for (int k = 0; k < topk; ++k) {
+      const int32_t row = __ldg(row_id_map + t * topk + k);
+      if (row < 0) continue;
+      q[((int64_t)row * ncb + j) * 8 + sub] = v[u];
+      if (sub == 0) sf[(int64_t)row * ncb + j] = e[u];
+    }
+  }
+}
+
 // grid (E, row slots): zero rows offsets[e] + totals[e] .. offsets[e+1]
 constexpr int kPadRowsPerCta = 8;
 __global__ void __launch_bounds__(256) pad_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ totals,
@@ -227,35 +268,52 @@ size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts
   return (size_t)(2 * C * num_experts + num_experts) * sizeof(int32_t) + 16;
 }
 
-fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,
-                                     const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
-                                     uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,
-                                     int32_t* row_id_map, void* workspace, cudaStream_t stream) {
-  (void)max_out_rows;
-  const int E = num_experts;
-  if (tokens == 0) {
-    return cudaMemsetAsync(expert_offsets, 0, (size_t)(E + 1) * sizeof(int32_t), stream) == cudaSuccess
-               ? FP8Q_OK
-               : FP8Q_ERR_CUDA;
-  }
+namespace {
+
+// Steps (1)-(3): offsets, per-chunk bases, row ids.
+fp8q_status route(const DeviceInfo& dev, int64_t tokens, const int32_t* topk_idx, int32_t topk, int E, int32_t align,
+                  int32_t* expert_offsets, int32_t* row_id_map, int32_t* counts, int32_t* bases, int32_t* totals,
+                  cudaStream_t stream) {
   const int64_t npairs = tokens * topk;
   const int64_t C = num_chunks(tokens, topk);
-  int32_t* counts = static_cast<int32_t*>(workspace);
-  int32_t* bases = counts + C * E;
-  int32_t* totals = bases + C * E;
   const size_t hist_smem = (size_t)E * sizeof(int32_t);
   count_kernel<<<(unsigned)C, 256, hist_smem, stream>>>(topk_idx, npairs, E, counts, dev.status);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   scan_kernel<<<1, 1024, 0, stream>>>(counts, C, E, align, expert_offsets, bases, totals);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   rank_kernel<<<(unsigned)C, 32, hist_smem, stream>>>(topk_idx, npairs, E, bases, row_id_map);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// xq/xsf != nullptr: FP8-input payload; else quantize x.
+fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq, const uint8_t* xsf, int64_t tokens,
+                        int64_t hidden, const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
+                        uint8_t* q, uint8_t* sf, int32_t* expert_offsets, int32_t* row_id_map, void* workspace,
+                        cudaStream_t stream) {
+  const int E = num_experts;
+  if (tokens == 0) {
+    return cudaMemsetAsync(expert_offsets, 0, (size_t)(E + 1) * sizeof(int32_t), stream) == cudaSuccess
+               ? FP8Q_OK
+               : FP8Q_ERR_CUDA;
+  }
+  const int64_t C = num_chunks(tokens, topk);
+  int32_t* counts = static_cast<int32_t*>(workspace);
+  int32_t* bases = counts + C * E;
+  int32_t* totals = bases + C * E;
+  const fp8q_status rs = route(dev, tokens, topk_idx, topk, E, align, expert_offsets, row_id_map, counts, bases,
+                               totals, stream);
+  if (rs != FP8Q_OK) return rs;
   if (hidden == 0) return FP8Q_OK;  // routing only: offsets and row ids, no payload
   const int ncb = (int)(hidden / 128);
   const int64_t n_tiles = tokens * ncb;
   const int64_t tiles_per_block = (kSThreads / 32) * kSUnroll * 4;
-  scatter_quant_kernel<<<(unsigned)((n_tiles + tiles_per_block - 1) / tiles_per_block), kSThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), tokens, ncb, row_id_map, topk, reinterpret_cast<uint2*>(q), sf);
+  const unsigned blocks = (unsigned)((n_tiles + tiles_per_block - 1) / tiles_per_block);
+  if (xq)
+    scatter_copy_kernel<<<blocks, kSThreads, 0, stream>>>(reinterpret_cast<const uint4*>(xq), xsf, tokens, ncb,
+                                                         row_id_map, topk, reinterpret_cast<uint4*>(q), sf);
+  else
+    scatter_quant_kernel<<<blocks, kSThreads, 0, stream>>>(static_cast<const uint4*>(x), tokens, ncb, row_id_map,
+                                                          topk, reinterpret_cast<uint2*>(q), sf);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   if (align > 1) {
     dim3 grid((unsigned)E, (unsigned)((align - 1 + kPadRowsPerCta - 1) / kPadRowsPerCta));
@@ -263,6 +321,27 @@ fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64
     if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   }
   return FP8Q_OK;
+}
+
+}  // namespace
+
+fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,
+                                     const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
+                                     uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,
+                                     int32_t* row_id_map, void* workspace, cudaStream_t stream) {
+  (void)max_out_rows;
+  return permute_pad(dev, x, nullptr, nullptr, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
+                     expert_offsets, row_id_map, workspace, stream);
+}
+
+fp8q_status launch_permute_pad_fp8(const DeviceInfo& dev, const uint8_t* xq, const uint8_t* xsf, int64_t tokens,
+                                   int64_t hidden, const int32_t* topk_idx, int32_t topk, int32_t num_experts,
+                                   int32_t align, uint8_t* q, uint8_t* sf, int64_t max_out_rows,
+                                   int32_t* expert_offsets, int32_t* row_id_map, void* workspace,
+                                   cudaStream_t stream) {
+  (void)max_out_rows;
+  return permute_pad(dev, nullptr, xq, xsf, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
+                     expert_offsets, row_id_map, workspace, stream);
 }
 
 }  // namespace fp8q

@@ -122,6 +122,26 @@ def test_packed_sf_bytes(L):
     assert sat.packed_sf_shape(3, 640) == (2, 4)
 
 
+def test_unpermute_host_errors(L):
+    f = L.fp8q_unpermute_unpad
+
+    def call(y=A, sf=None, rows=64, hidden=256, rmap=A, w=A, tokens=16, topk=2, out=A):
+        return f(y, sf, rows, hidden, rmap, w, tokens, topk, out, None)
+
+    assert call(hidden=200) == sat.FP8Q_ERR_SHAPE
+    assert call(rows=-1) == sat.FP8Q_ERR_SHAPE
+    assert call(topk=0) == sat.FP8Q_ERR_ARG
+    assert call(topk=65) == sat.FP8Q_ERR_ARG
+    assert call(y=None) == sat.FP8Q_ERR_NULL
+    assert call(rmap=None) == sat.FP8Q_ERR_NULL
+    assert call(out=None) == sat.FP8Q_ERR_NULL
+    assert call(y=MIS) == sat.FP8Q_ERR_ALIGN
+    assert call(out=MIS) == sat.FP8Q_ERR_ALIGN
+    assert call(rmap=A + 2) == sat.FP8Q_ERR_ALIGN
+    assert call(w=A + 1) == sat.FP8Q_ERR_ALIGN
+    assert call(y=None, rmap=None, out=None, tokens=0) == sat.FP8Q_OK   # empty: no-op
+
+
 def test_permute_host_errors(L):
     f = L.fp8q_permute_pad_quant
 
@@ -145,6 +165,28 @@ def test_permute_host_errors(L):
     assert call(x=None) == sat.FP8Q_ERR_NULL
     assert call(x=MIS) == sat.FP8Q_ERR_ALIGN
     assert call(rmap=A + 2) == sat.FP8Q_ERR_ALIGN
+
+
+def test_permute_fp8_host_errors(L):
+    f = L.fp8q_permute_pad_fp8
+
+    def call(tokens=16, hidden=256, topk=2, E=4, align=16, max_rows=None, ws=1 << 20, **kw):
+        if max_rows is None:
+            max_rows = tokens * topk + E * (align - 1)
+        p = dict(xq=A, xsf=A, idx=A, q=A, sf=A, off=A, rmap=A, wsp=A)
+        p.update(kw)
+        return f(p["xq"], p["xsf"], tokens, hidden, p["idx"], topk, E, align, p["q"], p["sf"], max_rows, p["off"],
+                 p["rmap"], p["wsp"], ws, None)
+
+    assert call(hidden=100) == sat.FP8Q_ERR_SHAPE
+    assert call(topk=0) == sat.FP8Q_ERR_ARG
+    assert call(max_rows=10) == sat.FP8Q_ERR_ARG
+    assert call(ws=4) == sat.FP8Q_ERR_ARG
+    assert call(xq=None) == sat.FP8Q_ERR_NULL
+    assert call(xsf=None) == sat.FP8Q_ERR_NULL
+    assert call(off=None) == sat.FP8Q_ERR_NULL
+    assert call(xq=MIS) == sat.FP8Q_ERR_ALIGN
+    assert call(q=MIS) == sat.FP8Q_ERR_ALIGN
 
 
 def test_binding_rejects_host_tensors():

@@ -132,3 +132,54 @@ def test_bounded_wait_expires_cleanly():
     x = dev(synthetic.scaled_normal(128, 128, seed=1))
     q, sf = sat.quantize_rowwise(x)
     device_status_ok()
+
+
+# ------------------------------------------------------------------ FP8-input permute
+
+def check_permute_fp8(x_bits, idx, E, align):
+    oq0, osf0 = oracle.quantize_rowwise(x_bits)
+    q, sf, off, rmap = sat.permute_pad_fp8(dev(oq0), dev(osf0), dev(idx), E, align)
+    device_status_ok()
+    oq, osf, ooff, ormap = oracle.permute_pad_fp8(oq0, osf0, idx, E, align)
+    assert_bytes_equal(host(off), ooff, "expert offsets")
+    assert_bytes_equal(host(rmap), ormap, "row_id_map")
+    n = int(ooff[-1])
+    assert_bytes_equal(host(sf)[:n], osf[:n], "SF")
+    assert_bytes_equal(host(q)[:n], oq[:n], "Q")
+    return q, sf, off
+
+
+@pytest.mark.parametrize("tokens,hidden,E,K,align", [(8, 128, 4, 2, 16), (100, 256, 8, 2, 16),
+                                                      (512, 384, 32, 8, 128), (3000, 256, 16, 4, 1),
+                                                      (1500, 512, 7, 3, 64)])
+def test_permute_fp8_shapes(tokens, hidden, E, K, align):
+    rng = np.random.default_rng(tokens + 5)
+    x = synthetic.scaled_normal(tokens, hidden, seed=tokens + 2)
+    check_permute_fp8(x, synthetic.zipf_topk(tokens, E, K, rng), E, align)
+
+
+def test_permute_fp8_equals_fused_permute_quantize_on_gpu():
+    """On the MoE workload: quantize on the GPU, permute the FP8 rows, and compare with the
+    fused BF16 permute+quantize - the same bytes in every written row."""
+    d = synthetic.moe()
+    x, idx = dev(d["x"]), dev(d["topk_idx"])
+    q0, sf0 = sat.quantize_rowwise(x)
+    a = sat.permute_pad_fp8(q0, sf0, idx, 32, 128)
+    b = sat.permute_pad_quant(x, idx, 32, 128)
+    device_status_ok()
+    n = int(b[2][-1].item())
+    assert torch.equal(a[2], b[2]) and torch.equal(a[3], b[3])
+    assert torch.equal(a[0][:n], b[0][:n]) and torch.equal(a[1][:n], b[1][:n])
+
+
+def test_permute_fp8_moe_config_full():
+    d = synthetic.moe()
+    check_permute_fp8(d["x"], d["topk_idx"], 32, 128)
+
+
+def test_permute_fp8_bad_index_sets_device_status():
+    q = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
+    sf = torch.full((4, 1), 127, dtype=torch.uint8, device="cuda")
+    idx = torch.tensor([[0], [1], [9], [2]], dtype=torch.int32, device="cuda")
+    sat.permute_pad_fp8(q, sf, idx, 4, 16)
+    assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE
