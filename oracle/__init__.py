@@ -67,6 +67,8 @@ def _declare(L):
         "orc_quantize_rowwise_colwise": [V, I64, I64, ctypes.c_uint32, V, V, V, V],
         "orc_unpermute_unpad": [V, V, I64, I64, V, V, I64, I32, V],
         "orc_permute_pad_fp8": [V, V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
+        "orc_quantize_rowwise_g": [V, I64, I64, I32, V, V],
+        "orc_direct_transpose_g": [V, V, I64, I64, I32, V, V],
     }.items():
         fn = getattr(L, name)
         fn.argtypes, fn.restype = args, ctypes.c_int
@@ -179,6 +181,29 @@ def quantize_rowwise_colwise(x_bf16_bits, flags: int = 0, colwise: bool = True):
     if rc:
         raise OracleError(f"oracle single-pass quantizer rejected its arguments (code {rc})")
     return q, sf, qt, sft
+
+
+def quantize_rowwise_g(x_bf16_bits, tile: int):
+    """Row-wise quantization with 1 x tile scaling tiles (tile = 128, or 32 for MX)."""
+    x = _c(x_bf16_bits, np.uint16)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // tile), np.uint8)
+    if lib().orc_quantize_rowwise_g(_p(x), rows, cols, tile, _p(q), _p(sf)):
+        raise OracleError("cols must be a multiple of the tile")
+    return q, sf
+
+
+def direct_transpose_g(q, sf, tile: int):
+    """Direct transpose with tile x tile blocks: (Q^T [cols, rows], SF^T [cols, rows/tile])."""
+    q = _c(q, np.uint8)
+    sf = _c(sf, np.uint8)
+    rows, cols = q.shape
+    qt = np.empty((cols, rows), np.uint8)
+    sft = np.empty((cols, rows // tile), np.uint8)
+    if lib().orc_direct_transpose_g(_p(q), _p(sf), rows, cols, tile, _p(qt), _p(sft)):
+        raise OracleError("rows and cols must be multiples of the tile")
+    return qt, sft
 
 
 def _transpose_common(fn, q, sf, offsets):

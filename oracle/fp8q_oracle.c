@@ -404,6 +404,67 @@ int orc_naive_transpose(const uint8_t *q, const uint8_t *sf, int64_t rows, int64
 }
 
 /* ------------------------------------------------------------------ */
+/* Tile size as a parameter: the 1x32 / 32x32 MX granularity            */
+/* ------------------------------------------------------------------ */
+
+/* [LP] format table: MXFP8 keeps E4M3 elements with one power-of-two (E8M0) scale per
+ * 32 elements; [FLOW] 局限与 Future Work 2 names the extension of the scaling-aware
+ * layout conversion to MX formats.  Reading: the same scale rule, on 1 x G tiles, and
+ * the same direct transpose on G x G blocks (G = 128 is the path above, G = 32 the MX
+ * granularity).  Layouts: SF [rows, cols/G], Q^T [cols, rows], SF^T [cols, rows/G].
+ * rows (for the transpose) and cols must be multiples of G.  Returns 0 or 2. */
+int orc_quantize_rowwise_g(const uint16_t *x, int64_t rows, int64_t cols, int32_t G, uint8_t *q, uint8_t *sf)
+{
+    if (G < 1 || G > 128 || cols % G)
+        return 2;
+    int64_t nt = cols / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < rows; t++)
+        for (int64_t j = 0; j < nt; j++) {
+            double amax = 0.0;
+            for (int i = 0; i < G; i++) {
+                double a = fabs(bf16_to_double(x[t * cols + j * G + i]));
+                if (a > amax)
+                    amax = a;
+            }
+            int e = orc_scale_exponent(amax);
+            for (int i = 0; i < G; i++)
+                q[t * cols + j * G + i] = orc_e4m3_encode(ldexp(bf16_to_double(x[t * cols + j * G + i]), -e));
+            sf[t * nt + j] = (uint8_t)(e + 127);
+        }
+    return 0;
+}
+
+int orc_direct_transpose_g(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t cols, int32_t G, uint8_t *qt,
+                           uint8_t *sft)
+{
+    if (G < 1 || G > 128 || cols % G || rows % G)
+        return 2;
+    int64_t nt = cols / G, nb = rows / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; b++)
+        for (int64_t j = 0; j < nt; j++) {
+            int emax = -1000;
+            for (int t = 0; t < G; t++) {
+                int e = (int)sf[(b * G + t) * nt + j] - 127;
+                if (e > emax)
+                    emax = e;
+            }
+            for (int t = 0; t < G; t++) {
+                int64_t row = b * G + t;
+                int k = emax - ((int)sf[row * nt + j] - 127);
+                for (int h = 0; h < G; h++) {
+                    int64_t ch = j * G + h;
+                    qt[ch * rows + row] = orc_shift_code_value(q[row * cols + ch], k);
+                }
+            }
+            for (int h = 0; h < G; h++)
+                sft[(j * G + h) * nb + b] = (uint8_t)(emax + 127);
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Single-pass quantization into both layouts, packed UE8M0 scales      */
 /* ------------------------------------------------------------------ */
 
