@@ -38,6 +38,8 @@ BYTES_QUANT = 2 * N_ELEM + N_ELEM + N_ELEM // 128            # read X, write Q +
 BYTES_DIRECT = N_ELEM + N_ELEM // 128 + N_ELEM + N_ELEM // 128  # read Q + SF, write Q^T + SF^T
 BYTES_STEP = BYTES_QUANT + BYTES_DIRECT
 BYTES_ROWCOL = 2 * N_ELEM + 2 * (N_ELEM + N_ELEM // 128)      # read X, write Q + SF + Q^T + SF^T
+BYTES_MX_QUANT = 3 * N_ELEM + N_ELEM // 32                      # 1x32 tiles
+BYTES_MX_DIRECT = 2 * (N_ELEM + N_ELEM // 32)                   # 32x32 blocks
 METRIC = "direct-transpose & quantize GB/s on 1 B200 (% of HBM peak); bit-exact vs oracle"
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
@@ -57,7 +59,8 @@ def measured_peak_gbs():
 def kernel_sources(kind: str):
     csrc = os.path.join(ROOT, "scaling_aware_transpose_b200", "csrc")
     main = {"quantize": "quantize_rowwise.cu", "direct": "direct_transpose.cu", "swiglu": "swiglu_quant.cu",
-            "permute": "permute_pad_quant.cu", "rowwise_colwise": "quantize_rowwise_colwise.cu"}[kind]
+            "permute": "permute_pad_quant.cu", "rowwise_colwise": "quantize_rowwise_colwise.cu",
+            "unpermute": "unpermute_unpad.cu", "mx32": "mx32.cu"}[kind]
     return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")]
 
 
@@ -409,6 +412,14 @@ def run_ours(args, rank, world, local_rank):
     t_rc = time_on_stream(rowcol, min(K, 50) + 3, stream, lambda: flush.fill_(10))
     t_rc_clean = time_on_stream(rowcol, min(K, 50) + 3, stream, clean_flush)
     t_rc_pk = time_on_stream(rowcol_pk, min(K, 50) + 3, stream, lambda: flush.fill_(11))
+    # MX granularity: 1x32 tiles and 32x32 transpose blocks on the same X
+    mq, msf = torch.empty_like(q), torch.empty((ROWS, COLS // 32), dtype=torch.uint8, device=device)
+    mqt, msft = torch.empty_like(qt), torch.empty((COLS, ROWS // 32), dtype=torch.uint8, device=device)
+    t_mxq = time_on_stream(lambda: sat.fp8q_quantize_rowwise_mx32(x, ROWS, COLS, mq, msf, sp), min(K, 50) + 3, stream,
+                           lambda: flush.fill_(15))
+    t_mxd = time_on_stream(lambda: sat.fp8q_direct_transpose_mx32(mq, msf, ROWS, COLS, mqt, msft, sp),
+                           min(K, 50) + 3, stream, lambda: flush.fill_(16))
+    del mq, msf, mqt, msft
     rowcol()
     torch.cuda.synchronize()
     same_rc = all(torch.equal(a_, b_) for a_, b_ in ((rc_q, q), (rc_sf, sf), (rc_qt, qt), (rc_sft, sft)))
@@ -478,6 +489,8 @@ def run_ours(args, rank, world, local_rank):
                 "vs_two_kernel_step": round((avg_q + avg_d) / t_rc, 3),
                 "outputs_equal_two_kernel_step": same_rc,
                 "traffic": profiled_traffic("rowwise_colwise")},
+            "mx32": {"quantize_us": round(t_mxq * 1e6, 2), "quantize_GB/s": round(BYTES_MX_QUANT / t_mxq / 1e9, 1),
+                     "direct_us": round(t_mxd * 1e6, 2), "direct_GB/s": round(BYTES_MX_DIRECT / t_mxd / 1e9, 1)},
             "clean_l2_flush": {"quantize_us": round(t_q_clean * 1e6, 2),
                                "quantize_GB/s": round(BYTES_QUANT / t_q_clean / 1e9, 1),
                                "direct_us": round(t_d_clean * 1e6, 2),

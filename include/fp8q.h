@@ -230,6 +230,23 @@ fp8q_status fp8q_permute_pad_fp8(const uint8_t *xq, const uint8_t *xsf, int64_t 
                                  int32_t *row_id_map, void *workspace, size_t workspace_bytes,
                                  fp8q_stream_t stream);
 
+/* The path at MX granularity (low-precision format table: MXFP8 = E4M3 elements with one
+ * power-of-two scale per 32 elements; FP8-Flow-MoE 局限与 Future Work 2: the
+ * scaling-aware conversion carried to MX formats).  Same scale rule and shift as above,
+ * with 1x32 scaling tiles and 32x32 transpose blocks.
+ *   fp8q_quantize_rowwise_mx32: x bf16 [rows, cols], cols % 32 == 0 -> q u8 [rows, cols],
+ *     sf u8 [rows, cols/32].  x and q 16-byte aligned.
+ *   fp8q_direct_transpose_mx32: (q, sf) as above -> qt u8 [cols, rows], sft u8
+ *     [cols, rows/32] holding, for channel h and token group g, the largest scale byte of
+ *     the 32x32 block (g, h/32).  This build's kernel needs rows % 128 == 0 and
+ *     cols % 128 == 0 (its CTA tile is 128x128, sixteen MX blocks).  q and qt 16-byte
+ *     aligned.
+ * Errors: NULL, ALIGN, SHAPE, CUDA. */
+fp8q_status fp8q_quantize_rowwise_mx32(const void *x, int64_t rows, int64_t cols, uint8_t *q, uint8_t *sf,
+                                       fp8q_stream_t stream);
+fp8q_status fp8q_direct_transpose_mx32(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t cols,
+                                       uint8_t *qt, uint8_t *sft, fp8q_stream_t stream);
+
 /* Size of the library's static scratch for fp8q_permute_pad_quant_noalloc (4 MiB). */
 #define FP8Q_NOALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
             "fp8q_permute_pad_fp8": ([P, P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
             "fp8q_permute_pad_quant_noalloc": ([P, I64, I64, P, I32, I32, I32, P, P, I64, P, P, P], ctypes.c_int),
             "fp8q_unpermute_unpad": ([P, P, I64, I64, P, P, I64, I32, P, P], ctypes.c_int),
+            "fp8q_quantize_rowwise_mx32": ([P, I64, I64, P, P, P], ctypes.c_int),
+            "fp8q_direct_transpose_mx32": ([P, P, I64, I64, P, P, P], ctypes.c_int),
             "fp8q_debug_expire_wait": ([ctypes.c_uint64, P], ctypes.c_int),
             "fp8q_version": ([], ctypes.c_int),
         }
@@ -188,6 +190,16 @@ def fp8q_unpermute_unpad(y, y_sf, rows: int, hidden: int, row_id_map, weights, t
                          stream=None) -> None:
     _check(lib().fp8q_unpermute_unpad(_ptr(y), _ptr(y_sf), rows, hidden, _ptr(row_id_map), _ptr(weights), tokens,
                                       topk, _ptr(out), _stream(stream)), "fp8q_unpermute_unpad")
+
+
+def fp8q_quantize_rowwise_mx32(x, rows: int, cols: int, q, sf, stream=None) -> None:
+    _check(lib().fp8q_quantize_rowwise_mx32(_ptr(x), rows, cols, _ptr(q), _ptr(sf), _stream(stream)),
+           "fp8q_quantize_rowwise_mx32")
+
+
+def fp8q_direct_transpose_mx32(q, sf, rows: int, cols: int, qt, sft, stream=None) -> None:
+    _check(lib().fp8q_direct_transpose_mx32(_ptr(q), _ptr(sf), rows, cols, _ptr(qt), _ptr(sft), _stream(stream)),
+           "fp8q_direct_transpose_mx32")
 
 
 def fp8q_debug_expire_wait(timeout_ns: int, stream=None) -> None:
@@ -333,3 +345,23 @@ def unpermute_unpad(y, row_id_map, topk: int, weights=None, y_sf=None, stream=No
     out = _empty((tokens, hidden), torch.bfloat16, y)
     fp8q_unpermute_unpad(y, y_sf, rows, hidden, row_id_map, weights, tokens, topk, out, stream)
     return out
+
+
+def quantize_rowwise_mx32(x, stream=None):
+    """1x32 tiles: (q [rows, cols], sf [rows, cols/32])."""
+    import torch
+    rows, cols = x.shape
+    q = _empty((rows, cols), torch.uint8, x)
+    sf = _empty((rows, cols // 32), torch.uint8, x)
+    fp8q_quantize_rowwise_mx32(x, rows, cols, q, sf, stream)
+    return q, sf
+
+
+def direct_transpose_mx32(q, sf, stream=None):
+    """32x32 blocks: (qt [cols, rows], sft [cols, rows/32])."""
+    import torch
+    rows, cols = q.shape
+    qt = _empty((cols, rows), torch.uint8, q)
+    sft = _empty((cols, rows // 32), torch.uint8, q)
+    fp8q_direct_transpose_mx32(q, sf, rows, cols, qt, sft, stream)
+    return qt, sft

@@ -249,6 +249,24 @@ fp8q_status fp8q_unpermute_unpad(const void* y, const uint8_t* y_sf, int64_t row
                                       as_stream(stream));
 }
 
+fp8q_status fp8q_quantize_rowwise_mx32(const void* x, int64_t rows, int64_t cols, uint8_t* q, uint8_t* sf,
+                                       fp8q_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 32 || rows > kMaxDim || cols > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  if (!x || !q || !sf) return FP8Q_ERR_NULL;
+  if (!aligned16(x) || !aligned16(q)) return FP8Q_ERR_ALIGN;
+  return fp8q::launch_quantize_mx32(x, rows, cols, q, sf, as_stream(stream));
+}
+
+fp8q_status fp8q_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols, uint8_t* qt,
+                                       uint8_t* sft, fp8q_stream_t stream) {
+  if (rows < 0 || cols < 0 || rows % 128 || cols % 128 || rows > kMaxDim || cols > kMaxDim) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  if (!q || !sf || !qt || !sft) return FP8Q_ERR_NULL;
+  if (!aligned16(q) || !aligned16(qt)) return FP8Q_ERR_ALIGN;
+  return fp8q::launch_direct_transpose_mx32(q, sf, rows, cols, qt, sft, as_stream(stream));
+}
+
 fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream) {
   if (timeout_ns < 1000ull) timeout_ns = 1000ull;
   if (timeout_ns > 2000000000ull) timeout_ns = 2000000000ull;

@@ -56,6 +56,11 @@ fp8q_status launch_permute_pad_fp8(const DeviceInfo& dev, const uint8_t* xq, con
                                    int32_t* expert_offsets, int32_t* row_id_map, void* workspace,
                                    cudaStream_t stream);
 
+fp8q_status launch_quantize_mx32(const void* x, int64_t rows, int64_t cols, uint8_t* q, uint8_t* sf,
+                                 cudaStream_t stream);
+fp8q_status launch_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols, uint8_t* qt,
+                                         uint8_t* sft, cudaStream_t stream);
+
 fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace fp8q

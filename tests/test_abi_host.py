@@ -142,6 +142,19 @@ def test_unpermute_host_errors(L):
     assert call(y=None, rmap=None, out=None, tokens=0) == sat.FP8Q_OK   # empty: no-op
 
 
+def test_mx32_host_errors(L):
+    fq, fd = L.fp8q_quantize_rowwise_mx32, L.fp8q_direct_transpose_mx32
+    assert fq(A, 4, 48, A, A, None) == sat.FP8Q_ERR_SHAPE          # cols % 32
+    assert fq(None, 4, 64, A, A, None) == sat.FP8Q_ERR_NULL
+    assert fq(MIS, 4, 64, A, A, None) == sat.FP8Q_ERR_ALIGN
+    assert fq(None, 0, 64, None, None, None) == sat.FP8Q_OK        # empty: no-op
+    assert fd(A, A, 96, 128, A, A, None) == sat.FP8Q_ERR_SHAPE     # rows % 128 (this build's kernel)
+    assert fd(A, A, 128, 160, A, A, None) == sat.FP8Q_ERR_SHAPE
+    assert fd(A, A, 128, 128, None, A, None) == sat.FP8Q_ERR_NULL
+    assert fd(A, A, 128, 128, MIS, A, None) == sat.FP8Q_ERR_ALIGN
+    assert fd(None, None, 0, 128, None, None, None) == sat.FP8Q_OK
+
+
 def test_permute_host_errors(L):
     f = L.fp8q_permute_pad_quant
 
