@@ -560,6 +560,17 @@ def run_profile(args):
             "naive": lambda: sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, ws, ws.numel()),
             "rowwise_colwise": lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, 0, q, sf, qt, sft),
         }
+    elif args.profile == "mx32":
+        x = synthetic.to_torch_bf16(synthetic.dense(seed=0)["x"]).cuda()
+        mq, msf = sat.quantize_rowwise_mx32(x)
+        mqt, msft = sat.direct_transpose_mx32(mq, msf)
+        calls = {"mx32": lambda: sat.fp8q_direct_transpose_mx32(mq, msf, ROWS, COLS, mqt, msft)}
+    elif args.profile == "permute_fp8":
+        d = synthetic.moe()
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        xq, xsf = sat.quantize_rowwise(x)
+        calls = {"permute_fp8": lambda: sat.permute_pad_fp8(xq, xsf, idx, d["num_experts"], 128)}
     elif args.profile == "swiglu":
         d = synthetic.swiglu()
         g, u = synthetic.to_torch_bf16(d["gate"]).cuda(), synthetic.to_torch_bf16(d["up"]).cuda()
@@ -605,7 +616,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
     ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise",
-                                          "unpermute"],
+                                          "unpermute", "mx32", "permute_fp8"],
                     default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)

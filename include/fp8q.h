@@ -240,7 +240,7 @@ fp8q_status fp8q_permute_pad_fp8(const uint8_t *xq, const uint8_t *xsf, int64_t 
  *     [cols, rows/32] holding, for channel h and token group g, the largest scale byte of
  *     the 32x32 block (g, h/32).  This build's kernel needs rows % 128 == 0 and
  *     cols % 128 == 0 (its CTA tile is 128x128, sixteen MX blocks).  q and qt 16-byte
- *     aligned.
+ *     aligned, sf and sft 4-byte aligned.
  * Errors: NULL, ALIGN, SHAPE, CUDA. */
 fp8q_status fp8q_quantize_rowwise_mx32(const void *x, int64_t rows, int64_t cols, uint8_t *q, uint8_t *sf,
                                        fp8q_stream_t stream);

@@ -263,7 +263,8 @@ fp8q_status fp8q_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, int6
   if (rows < 0 || cols < 0 || rows % 128 || cols % 128 || rows > kMaxDim || cols > kMaxDim) return FP8Q_ERR_SHAPE;
   if (rows == 0 || cols == 0) return FP8Q_OK;
   if (!q || !sf || !qt || !sft) return FP8Q_ERR_NULL;
-  if (!aligned16(q) || !aligned16(qt)) return FP8Q_ERR_ALIGN;
+  if (!aligned16(q) || !aligned16(qt) || (reinterpret_cast<uintptr_t>(sf) & 3u) || (reinterpret_cast<uintptr_t>(sft) & 3u))
+    return FP8Q_ERR_ALIGN;
   return fp8q::launch_direct_transpose_mx32(q, sf, rows, cols, qt, sft, as_stream(stream));
 }
 

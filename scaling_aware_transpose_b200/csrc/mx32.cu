@@ -14,10 +14,11 @@
 // and stores 8 codes per chunk (256 contiguous bytes per store instruction).
 //
 // direct_transpose_mx32_kernel: the 128x128 block-per-CTA direct transpose with 16 MX
-// blocks per CTA tile.  Each row holds four scale bytes (one per 32-column group); warp
-// w reduces Smax of row group w for all four column groups at once with a packed
-// byte-wise max (__vmaxu4) over five shuffles.  The shift of a 16-byte row chunk uses
-// its own 32x32 block's k; staging and the byte transpose are those of the 128 kernel.
+// blocks per CTA tile.  Each row's four scale bytes (one per 32-column group) move as one
+// 32-bit word; every warp reduces the packed Smax words of all four row groups itself
+// (a byte-wise max, __vmaxu4, over five shuffles each, the four chains interleaved), so
+// one barrier suffices as in the 128 kernel.  The shift of a 16-byte row chunk uses its
+// own 32x32 block's k; staging and the byte transpose are those of the 128 kernel.
 #include "common.cuh"
 #include "launch.h"
 
@@ -70,14 +71,19 @@ constexpr int kPasses = 4;
 
 __device__ __forceinline__ int chunk_pos(int r, int c) { return c ^ ((r >> 4) & 7); }
 __device__ __forceinline__ int byte_of(uint32_t w, int i) { return (int)((w >> (8 * i)) & 0xFFu); }
+// Byte c of each of four words, packed (word i -> byte i).
+__device__ __forceinline__ uint32_t gather_byte4(const uint32_t (&w)[4], int c) {
+  const uint32_t lo = __byte_perm(w[0], w[1], (uint32_t)(c | ((c + 4) << 4)));
+  const uint32_t hi = __byte_perm(w[2], w[3], (uint32_t)(c | ((c + 4) << 4)));
+  return __byte_perm(lo, hi, 0x5410);
+}
 
-__global__ void __launch_bounds__(kThreads, 8) direct_transpose_mx32_kernel(const uint8_t* __restrict__ q,
+__global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(const uint8_t* __restrict__ q,
                                                                           const uint8_t* __restrict__ sf, int64_t rows,
                                                                           int cols, uint8_t* __restrict__ qt,
                                                                           uint8_t* __restrict__ sft) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ uint32_t e_row[128];  // 4 scale bytes of the row: column groups 0..3 of this tile
-  __shared__ uint32_t e_max[4];    // per row group: packed Smax bytes of column groups 0..3
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const int ngr = cols >> 5;  // scale bytes per row
@@ -90,25 +96,26 @@ __global__ void __launch_bounds__(kThreads, 8) direct_transpose_mx32_kernel(cons
   uint4 v[kPasses];
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) v[p] = __ldg(reinterpret_cast<const uint4*>(qb + (p * 32 + rsub) * cols) + sub);
-  if (tid < 128) {
-    const uint8_t* s = sf + (r0 + tid) * ngr + (c0 >> 5);
-    e_row[tid] = (uint32_t)__ldg(s) | ((uint32_t)__ldg(s + 1) << 8) | ((uint32_t)__ldg(s + 2) << 16) |
-                 ((uint32_t)__ldg(s + 3) << 24);
-  }
+  // the row's 4 scale bytes: 4-byte aligned (rows of cols/32 bytes, cols % 128 == 0)
+  if (tid < 128) e_row[tid] = __ldg(reinterpret_cast<const uint32_t*>(sf + (r0 + tid) * ngr + (c0 >> 5)));
   __syncthreads();
-  if (tid < 128) {
-    uint32_t m = e_row[tid];
+  uint32_t e_max[4];  // per row group: packed Smax bytes of column groups 0..3
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = __vmaxu4(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if ((tid & 31) == 0) e_max[tid >> 5] = m;
-  }
-  __syncthreads();
+  for (int rg = 0; rg < 4; ++rg) e_max[rg] = e_row[32 * rg + (tid & 31)];
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+    for (int rg = 0; rg < 4; ++rg) e_max[rg] = __vmaxu4(e_max[rg], __shfl_xor_sync(0xFFFFFFFFu, e_max[rg], o));
+  // byte i of smax_mine: Smax of (row group i, this thread's column group); of smax_sft:
+  // Smax of (row group i, column group of channel c0 + tid) for the SF^T word
+  const int cg = sub >> 1;  // 32-column group of this thread's 16-byte chunks
+  const uint32_t smax_mine = gather_byte4(e_max, cg);
+  const uint32_t smax_sft = gather_byte4(e_max, (tid >> 5) & 3);
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
     const int rl = p * 32 + rsub;  // row group p
-    const int cg = sub >> 1;       // 32-column group of this 16-byte chunk
     uint32_t w[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
-    shift_row16(w, byte_of(e_max[p], cg) - byte_of(e_row[rl], cg));
+    shift_row16(w, byte_of(smax_mine, p) - byte_of(e_row[rl], cg));
     *reinterpret_cast<uint4*>(tile + rl * 128 + 16 * chunk_pos(rl, sub)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   __syncthreads();
@@ -128,12 +135,8 @@ __global__ void __launch_bounds__(kThreads, 8) direct_transpose_mx32_kernel(cons
 #pragma unroll
   for (int c = 0; c < 4; ++c, out += rows)
     *reinterpret_cast<uint4*>(out) = make_uint4(ov[c][0], ov[c][1], ov[c][2], ov[c][3]);
-  if (tid < 128) {  // SF^T [cols, rows/32]: channel c0 + tid, token groups 4b..4b+3
-    const int cg = tid >> 5;
-    uint8_t* d = sft + (int64_t)(c0 + tid) * (rows >> 5) + (r0 >> 5);
-#pragma unroll
-    for (int rg = 0; rg < 4; ++rg) d[rg] = (uint8_t)byte_of(e_max[rg], cg);
-  }
+  if (tid < 128)  // SF^T [cols, rows/32]: channel c0 + tid, token groups 4b..4b+3, one word
+    *reinterpret_cast<uint32_t*>(sft + (int64_t)(c0 + tid) * (rows >> 5) + (r0 >> 5)) = smax_sft;
 }
 
 }  // namespace

@@ -152,6 +152,8 @@ def test_mx32_host_errors(L):
     assert fd(A, A, 128, 160, A, A, None) == sat.FP8Q_ERR_SHAPE
     assert fd(A, A, 128, 128, None, A, None) == sat.FP8Q_ERR_NULL
     assert fd(A, A, 128, 128, MIS, A, None) == sat.FP8Q_ERR_ALIGN
+    assert fd(A, A + 2, 128, 128, A, A, None) == sat.FP8Q_ERR_ALIGN      # scale words
+    assert fd(A, A, 128, 128, A, A + 1, None) == sat.FP8Q_ERR_ALIGN
     assert fd(None, None, 0, 128, None, None, None) == sat.FP8Q_OK
 
 
