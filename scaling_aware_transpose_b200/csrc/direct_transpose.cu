@@ -8,7 +8,7 @@
 // transposed (1x128 along tokens) layout; §5.6: expert groups are contiguous row ranges.
 //
 // One CTA per 128x128 block, blocks in row-major order (column blocks fastest), eight
-// CTAs per SM (32 registers, 16.5 KB of shared memory each), so the CTAs resident at any
+// CTAs per SM (32 registers, 16.5 KB of shared memory each; six in grouped mode), so the CTAs resident at any
 // moment read a compact band of whole rows of Q and write runs of a few hundred bytes
 // into every row of Q^T; many small independent CTAs keep enough loads in flight
 // without a pipeline.  256 threads:
@@ -18,9 +18,9 @@
 //      exponent subtract when exact for all 16 bytes, else the f16 route, see
 //      shift_row16) and stored to a 16 KB tile whose 16-byte chunks are XOR-swizzled by
 //      row;
-//   3. each lane gathers 16 tokens x 4 channels with conflict-free 4-byte shared loads,
-//      transposes them with byte permutes and writes four 16-byte runs of Q^T (each warp
-//      store fills 128 bytes of four channel rows).
+//   3. each lane gathers 8 tokens x 8 channels with 8-byte shared loads (conflict-free per
+//      half-warp), transposes them with byte permutes (four 4x4 transposes) and writes
+//      eight 8-byte runs of Q^T (each warp store fills 128 bytes of two channel rows).
 // Grouped mode (expert offsets on the device): the grid covers the buffer's capacity;
 // each CTA finds its group by binary search, CTAs past the last group exit, and every
 // inconsistency is recorded in the status word instead of producing an address.
@@ -33,12 +33,12 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kPasses = 4;
 
-// Chunk c of tile row r sits at chunk position c ^ (r >> 4): the phase-3 reads of rows
-// 16t + i (t = 0..7) hit 8 distinct chunk positions.
-__device__ __forceinline__ int chunk_pos(int r, int c) { return c ^ ((r >> 4) & 7); }
+// Chunk c of tile row r sits at chunk position c ^ ((r >> 3) & 7): the phase-3 reads of
+// rows 8t + i (t = 0..7 in each half-warp) hit 8 distinct chunk positions.
+__device__ __forceinline__ int chunk_pos(int r, int c) { return c ^ ((r >> 3) & 7); }
 
 template <bool kGrouped>
-__global__ void __launch_bounds__(kThreads, 8) direct_transpose_kernel(const uint8_t* __restrict__ q,
+__global__ void __launch_bounds__(kThreads, kGrouped ? 6 : 8) direct_transpose_kernel(const uint8_t* __restrict__ q,
                                                                      const uint8_t* __restrict__ sf, int64_t rows,
                                                                      int cols, const int32_t* __restrict__ off,
                                                                      int G, uint8_t* __restrict__ qt,
@@ -83,23 +83,28 @@ __global__ void __launch_bounds__(kThreads, 8) direct_transpose_kernel(const uin
     *reinterpret_cast<uint4*>(tile + rl * 128 + 16 * chunk_pos(rl, sub)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   __syncthreads();
-  // ---- 3. transpose
+  // ---- 3. transpose (8 tokens x 8 channels per lane)
   const int lane = tid & 31, wi = tid >> 5;
-  const int t = lane >> 2, g = lane & 3;
-  uint32_t col[16];
+  const int t = lane >> 1, g = lane & 1;
+  uint32_t lo[8], hi[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int rl = 16 * t + i;
-    col[i] = *reinterpret_cast<const uint32_t*>(tile + rl * 128 + 16 * chunk_pos(rl, wi) + 4 * g);
+  for (int i = 0; i < 8; ++i) {
+    const int rl = 8 * t + i;
+    const uint2 w = *reinterpret_cast<const uint2*>(tile + rl * 128 + 16 * chunk_pos(rl, wi) + 8 * g);
+    lo[i] = w.x;
+    hi[i] = w.y;
   }
-  uint32_t ov[4][4];
+  uint32_t a[4][2], c[4][2];  // channel c (0..3 from lo, 4..7 from hi) x token quad
 #pragma unroll
-  for (int qd = 0; qd < 4; ++qd)
-    transpose4x4(col[4 * qd], col[4 * qd + 1], col[4 * qd + 2], col[4 * qd + 3], ov[0][qd], ov[1][qd], ov[2][qd], ov[3][qd]);
-  uint8_t* out = qt + cols * o + (int64_t)(c0 + 16 * wi + 4 * g) * M + (r0 - o) + 16 * t;
+  for (int qd = 0; qd < 2; ++qd) {
+    transpose4x4(lo[4 * qd], lo[4 * qd + 1], lo[4 * qd + 2], lo[4 * qd + 3], a[0][qd], a[1][qd], a[2][qd], a[3][qd]);
+    transpose4x4(hi[4 * qd], hi[4 * qd + 1], hi[4 * qd + 2], hi[4 * qd + 3], c[0][qd], c[1][qd], c[2][qd], c[3][qd]);
+  }
+  uint8_t* out = qt + cols * o + (int64_t)(c0 + 16 * wi + 8 * g) * M + (r0 - o) + 8 * t;
 #pragma unroll
-  for (int c = 0; c < 4; ++c, out += M)
-    *reinterpret_cast<uint4*>(out) = make_uint4(ov[c][0], ov[c][1], ov[c][2], ov[c][3]);
+  for (int k = 0; k < 4; ++k, out += M) *reinterpret_cast<uint2*>(out) = make_uint2(a[k][0], a[k][1]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k, out += M) *reinterpret_cast<uint2*>(out) = make_uint2(c[k][0], c[k][1]);
   if (tid < 128) sft[cols * o / 128 + (int64_t)(c0 + tid) * (M >> 7) + ((r0 - o) >> 7)] = (uint8_t)emax;
 }
 

@@ -18,7 +18,8 @@
 // 32-bit word; every warp reduces the packed Smax words of all four row groups itself
 // (a byte-wise max, __vmaxu4, over five shuffles each, the four chains interleaved), so
 // one barrier suffices as in the 128 kernel.  The shift of a 16-byte row chunk uses its
-// own 32x32 block's k; staging and the byte transpose are those of the 128 kernel.
+// own 32x32 block's k; staging and the byte transpose (8 tokens x 8 channels per lane)
+// are those of the 128 kernel.
 #include "common.cuh"
 #include "launch.h"
 
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_mx32_kernel(const uint4* _
 constexpr int kThreads = 256;
 constexpr int kPasses = 4;
 
-__device__ __forceinline__ int chunk_pos(int r, int c) { return c ^ ((r >> 4) & 7); }
+__device__ __forceinline__ int chunk_pos(int r, int c) { return c ^ ((r >> 3) & 7); }
 __device__ __forceinline__ int byte_of(uint32_t w, int i) { return (int)((w >> (8 * i)) & 0xFFu); }
 // Byte c of each of four words, packed (word i -> byte i).
 __device__ __forceinline__ uint32_t gather_byte4(const uint32_t (&w)[4], int c) {
@@ -120,21 +121,26 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   }
   __syncthreads();
   const int lane = tid & 31, wi = tid >> 5;
-  const int t = lane >> 2, g = lane & 3;
-  uint32_t col[16];
+  const int t = lane >> 1, g = lane & 1;  // 8 tokens x 8 channels per lane
+  uint32_t lo[8], hi[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int rl = 16 * t + i;
-    col[i] = *reinterpret_cast<const uint32_t*>(tile + rl * 128 + 16 * chunk_pos(rl, wi) + 4 * g);
+  for (int i = 0; i < 8; ++i) {
+    const int rl = 8 * t + i;
+    const uint2 w = *reinterpret_cast<const uint2*>(tile + rl * 128 + 16 * chunk_pos(rl, wi) + 8 * g);
+    lo[i] = w.x;
+    hi[i] = w.y;
   }
-  uint32_t ov[4][4];
+  uint32_t a[4][2], c[4][2];
 #pragma unroll
-  for (int qd = 0; qd < 4; ++qd)
-    transpose4x4(col[4 * qd], col[4 * qd + 1], col[4 * qd + 2], col[4 * qd + 3], ov[0][qd], ov[1][qd], ov[2][qd], ov[3][qd]);
-  uint8_t* out = qt + (int64_t)(c0 + 16 * wi + 4 * g) * rows + r0 + 16 * t;
+  for (int qd = 0; qd < 2; ++qd) {
+    transpose4x4(lo[4 * qd], lo[4 * qd + 1], lo[4 * qd + 2], lo[4 * qd + 3], a[0][qd], a[1][qd], a[2][qd], a[3][qd]);
+    transpose4x4(hi[4 * qd], hi[4 * qd + 1], hi[4 * qd + 2], hi[4 * qd + 3], c[0][qd], c[1][qd], c[2][qd], c[3][qd]);
+  }
+  uint8_t* out = qt + (int64_t)(c0 + 16 * wi + 8 * g) * rows + r0 + 8 * t;
 #pragma unroll
-  for (int c = 0; c < 4; ++c, out += rows)
-    *reinterpret_cast<uint4*>(out) = make_uint4(ov[c][0], ov[c][1], ov[c][2], ov[c][3]);
+  for (int k = 0; k < 4; ++k, out += rows) *reinterpret_cast<uint2*>(out) = make_uint2(a[k][0], a[k][1]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k, out += rows) *reinterpret_cast<uint2*>(out) = make_uint2(c[k][0], c[k][1]);
   if (tid < 128)  // SF^T [cols, rows/32]: channel c0 + tid, token groups 4b..4b+3, one word
     *reinterpret_cast<uint32_t*>(sft + (int64_t)(c0 + tid) * (rows >> 5) + (r0 >> 5)) = smax_sft;
 }

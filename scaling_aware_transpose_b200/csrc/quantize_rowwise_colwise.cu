@@ -15,9 +15,9 @@
 //   2. once the block's 128 exponents are in shared memory each warp reduces Smax, then
 //      encodes the row-wise codes, stores them with their scale, shifts them by the row's
 //      k (uniform over a thread's 16 codes) and stages them in a swizzled 16 KB tile;
-//   3. each lane gathers 16 tokens x 4 channels from the tile, transposes them with byte
-//      permutes and writes four 16-byte runs of Q^T (each warp store fills 128 bytes of
-//      four channel rows).
+//   3. each lane gathers 8 tokens x 8 channels from the tile, transposes them with byte
+//      permutes and writes eight 8-byte runs of Q^T (each warp store fills 128 bytes of
+//      two channel rows).
 // Options: an all-zero tile may take e = -127 instead of 0 (it then never raises Smax);
 // scales may be written as packed UE8M0 words (four K-consecutive scale bytes per
 // 32-bit word, MN-major: word (g, m) at g * mn_pad + m), the layout the SM100 GEMM reads
@@ -31,12 +31,12 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kPasses = 4;  // 4 passes x 32 rows; 8 lanes per 1x128 row tile
 
-// 16-byte chunk position of chunk `c` of tile row `r`.  Phase 2 reads one 4-byte word
-// from rows 16t + i (t = 0..7) of the same chunk: the (r >> 4) term spreads those over 8
-// distinct chunks.  Phase 1 writes 8-byte pieces of 4 consecutive rows, served per
-// half-warp (two rows each): the (r & 1) term puts the two rows of a half-warp into
+// 16-byte chunk position of chunk `c` of tile row `r`.  Phase 3 reads 8 bytes from rows
+// 8t + i (t = 0..7 in each half-warp) of the same chunk: the (r >> 3) term spreads those
+// over 8 distinct chunks.  Phase 2 writes 8-byte pieces of 4 consecutive rows, served
+// per half-warp (two rows each): the (r & 1) term puts the two rows of a half-warp into
 // opposite bank halves, so each 256-byte warp store takes the minimum two wavefronts.
-__device__ __forceinline__ int tile_chunk(int r, int c) { return c ^ ((r >> 4) & 7) ^ ((r & 1) << 2); }
+__device__ __forceinline__ int tile_chunk(int r, int c) { return c ^ ((r >> 3) & 7) ^ ((r & 1) << 2); }
 
 // Byte `i` (0..3) of packed scale word `word` := v; bytes are the K order of the tiles.
 __device__ __forceinline__ void put_packed(uint8_t* packed, int64_t word, int i, uint8_t v) { packed[word * 4 + i] = v; }
@@ -126,24 +126,29 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
   if (!kColwise) return;
 
-  // ---- 3. transpose: warp wi owns channels 16wi..16wi+15, lane (t, g) tokens 16t.. x 4 channels
+  // ---- 3. transpose: warp wi owns channels 16wi..16wi+15, lane (t, g) tokens 8t.. x 8 channels
   __syncthreads();
   const int lane = tid & 31, wi = tid >> 5;
-  const int t = lane >> 2, g = lane & 3;
-  uint32_t col[16];
+  const int t = lane >> 1, g = lane & 1;
+  uint32_t lo[8], hi[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int rl = 16 * t + i;
-    col[i] = *reinterpret_cast<const uint32_t*>(tile + rl * 128 + 16 * tile_chunk(rl, wi) + 4 * g);
+  for (int i = 0; i < 8; ++i) {
+    const int rl = 8 * t + i;
+    const uint2 w = *reinterpret_cast<const uint2*>(tile + rl * 128 + 16 * tile_chunk(rl, wi) + 8 * g);
+    lo[i] = w.x;
+    hi[i] = w.y;
   }
-  uint32_t o[4][4];  // [channel][token quad]
+  uint32_t a[4][2], c[4][2];  // [channel][token quad]: channels 0..3 from lo, 4..7 from hi
 #pragma unroll
-  for (int qd = 0; qd < 4; ++qd)
-    transpose4x4(col[4 * qd], col[4 * qd + 1], col[4 * qd + 2], col[4 * qd + 3], o[0][qd], o[1][qd], o[2][qd], o[3][qd]);
-  uint8_t* out = qt + (int64_t)(c0 + 16 * wi + 4 * g) * rows + r0 + 16 * t;
+  for (int qd = 0; qd < 2; ++qd) {
+    transpose4x4(lo[4 * qd], lo[4 * qd + 1], lo[4 * qd + 2], lo[4 * qd + 3], a[0][qd], a[1][qd], a[2][qd], a[3][qd]);
+    transpose4x4(hi[4 * qd], hi[4 * qd + 1], hi[4 * qd + 2], hi[4 * qd + 3], c[0][qd], c[1][qd], c[2][qd], c[3][qd]);
+  }
+  uint8_t* out = qt + (int64_t)(c0 + 16 * wi + 8 * g) * rows + r0 + 8 * t;
 #pragma unroll
-  for (int c = 0; c < 4; ++c, out += rows)
-    *reinterpret_cast<uint4*>(out) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+  for (int k = 0; k < 4; ++k, out += rows) *reinterpret_cast<uint2*>(out) = make_uint2(a[k][0], a[k][1]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k, out += rows) *reinterpret_cast<uint2*>(out) = make_uint2(c[k][0], c[k][1]);
 
   if (tid < 128) {
     const int64_t h = c0 + tid;
