@@ -10,10 +10,11 @@
 //
 // Launches: (1) per-chunk expert histograms, (2) one CTA scans them into padded expert
 // offsets and per-chunk bases, (3) one warp per chunk assigns stable ranks with
-// __match_any_sync, (4) the streaming scatter-quantize over all (token, tile) pairs,
-// (5) zero-fill of the padding rows.  Workspace: counts[C][E], bases[C][E], totals[E].
+// __match_any_sync, (4) the streaming scatter-quantize over all (token, tile) pairs, whose
+// trailing CTAs zero-fill the padding rows.  Workspace: counts[C][E], bases[C][E], totals[E].
 // The FP8-input variant (the dispatch already delivered row-wise codes and scales) shares
-// (1)-(3) and (5); its step (4) copies each token's codes and scale bytes to its rows.
+// (1)-(3) and the padding; its step (4) copies each token's codes and scale bytes to its
+// rows.
 #include "common.cuh"
 #include "launch.h"
 
@@ -157,6 +158,26 @@ __device__ __forceinline__ uint32_t encode4(uint32_t a, uint32_t b, float s) {
   return __byte_perm(cvt_e4m3x2_f32(f0, f1), cvt_e4m3x2_f32(f2, f3), 0x5410);
 }
 
+// Padding rows: CTA slot `slot` of expert e zeroes rows offsets[e] + totals[e] + 8*slot ..
+// (at most 8 rows, never past offsets[e+1]): codes 0x00, scale byte 127.  Run by the
+// trailing CTAs of the scatter launch (E x ceil((align-1)/8) of them).
+constexpr int kPadRowsPerCta = 8;
+__device__ __forceinline__ void pad_rows(int64_t pad_cta, int pad_slots, const int32_t* __restrict__ offsets,
+                                         const int32_t* __restrict__ totals, int64_t hidden, uint8_t* __restrict__ q,
+                                         uint8_t* __restrict__ sf) {
+  const int e = (int)(pad_cta / pad_slots);
+  const int slot = (int)(pad_cta - (int64_t)e * pad_slots);
+  const int64_t start = (int64_t)offsets[e] + totals[e], end = offsets[e + 1];
+  const int64_t ncb = hidden >> 7;
+  for (int rr = 0; rr < kPadRowsPerCta; ++rr) {
+    const int64_t r = start + (int64_t)slot * kPadRowsPerCta + rr;
+    if (r >= end) return;
+    uint4* row = reinterpret_cast<uint4*>(q + r * hidden);
+    for (int64_t i = threadIdx.x; i < hidden / 16; i += blockDim.x) row[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t i = threadIdx.x; i < ncb; i += blockDim.x) sf[r * ncb + i] = 127;
+  }
+}
+
 constexpr int kSThreads = 256;
 constexpr int kSUnroll = 2;
 
@@ -165,7 +186,15 @@ constexpr int kSUnroll = 2;
 // and quantized once and its codes written to the token's top-k destination rows.
 __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* __restrict__ x, int64_t tokens, int ncb,
                                                                   const int32_t* __restrict__ row_id_map, int topk,
-                                                                  uint2* __restrict__ q, uint8_t* __restrict__ sf) {
+                                                                  uint2* __restrict__ q, uint8_t* __restrict__ sf,
+                                                                  int64_t scatter_ctas, int pad_slots,
+                                                                  const int32_t* __restrict__ offsets,
+                                                                  const int32_t* __restrict__ totals) {
+  if ((int64_t)blockIdx.x >= scatter_ctas) {
+    pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
+             reinterpret_cast<uint8_t*>(q), sf);
+    return;
+  }
   const int lane = threadIdx.x & 31, sub = lane & 7;
   const int64_t n_tiles = tokens * ncb;
   const int64_t warp = ((int64_t)blockIdx.x * kSThreads + threadIdx.x) >> 5;
@@ -214,7 +243,14 @@ __global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __
                                                                  const uint8_t* __restrict__ xsf, int64_t tokens,
                                                                  int ncb, const int32_t* __restrict__ row_id_map,
                                                                  int topk, uint4* __restrict__ q,
-                                                                 uint8_t* __restrict__ sf) {
+                                                                 uint8_t* __restrict__ sf, int64_t scatter_ctas,
+                                                                 int pad_slots, const int32_t* __restrict__ offsets,
+                                                                 const int32_t* __restrict__ totals) {
+  if ((int64_t)blockIdx.x >= scatter_ctas) {
+    pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
+             reinterpret_cast<uint8_t*>(q), sf);
+    return;
+  }
   const int lane = threadIdx.x & 31, sub = lane & 7;
   const int64_t n_tiles = tokens * ncb;
   const int64_t warp = ((int64_t)blockIdx.x * kSThreads + threadIdx.x) >> 5;
@@ -242,22 +278,6 @@ __global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __
       q[((int64_t)row * ncb + j) * 8 + sub] = v[u];
       if (sub == 0) sf[(int64_t)row * ncb + j] = e[u];
     }
-  }
-}
-
-// grid (E, row slots): zero rows offsets[e] + totals[e] .. offsets[e+1]
-constexpr int kPadRowsPerCta = 8;
-__global__ void __launch_bounds__(256) pad_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ totals,
-                                                  int64_t hidden, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
-  const int e = blockIdx.x;
-  const int64_t start = (int64_t)offsets[e] + totals[e], end = offsets[e + 1];
-  const int64_t ncb = hidden >> 7;
-  for (int rr = 0; rr < kPadRowsPerCta; ++rr) {
-    const int64_t r = start + (int64_t)blockIdx.y * kPadRowsPerCta + rr;
-    if (r >= end) return;
-    uint4* row = reinterpret_cast<uint4*>(q + r * hidden);
-    for (int64_t i = threadIdx.x; i < hidden / 16; i += blockDim.x) row[i] = make_uint4(0u, 0u, 0u, 0u);
-    for (int64_t i = threadIdx.x; i < ncb; i += blockDim.x) sf[r * ncb + i] = 127;
   }
 }
 
@@ -307,20 +327,19 @@ fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq,
   const int ncb = (int)(hidden / 128);
   const int64_t n_tiles = tokens * ncb;
   const int64_t tiles_per_block = (kSThreads / 32) * kSUnroll * 4;
-  const unsigned blocks = (unsigned)((n_tiles + tiles_per_block - 1) / tiles_per_block);
+  const int64_t scatter_ctas = (n_tiles + tiles_per_block - 1) / tiles_per_block;
+  const int pad_slots = (align - 1 + kPadRowsPerCta - 1) / kPadRowsPerCta;  // 0 when align == 1
+  const int64_t blocks = scatter_ctas + (int64_t)E * pad_slots;
+  if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   if (xq)
-    scatter_copy_kernel<<<blocks, kSThreads, 0, stream>>>(reinterpret_cast<const uint4*>(xq), xsf, tokens, ncb,
-                                                         row_id_map, topk, reinterpret_cast<uint4*>(q), sf);
+    scatter_copy_kernel<<<(unsigned)blocks, kSThreads, 0, stream>>>(
+        reinterpret_cast<const uint4*>(xq), xsf, tokens, ncb, row_id_map, topk, reinterpret_cast<uint4*>(q), sf,
+        scatter_ctas, pad_slots, expert_offsets, totals);
   else
-    scatter_quant_kernel<<<blocks, kSThreads, 0, stream>>>(static_cast<const uint4*>(x), tokens, ncb, row_id_map,
-                                                          topk, reinterpret_cast<uint2*>(q), sf);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  if (align > 1) {
-    dim3 grid((unsigned)E, (unsigned)((align - 1 + kPadRowsPerCta - 1) / kPadRowsPerCta));
-    pad_kernel<<<grid, 256, 0, stream>>>(expert_offsets, totals, hidden, q, sf);
-    if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  }
-  return FP8Q_OK;
+    scatter_quant_kernel<<<(unsigned)blocks, kSThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), tokens, ncb, row_id_map, topk, reinterpret_cast<uint2*>(q), sf, scatter_ctas,
+        pad_slots, expert_offsets, totals);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 }  // namespace
