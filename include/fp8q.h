@@ -281,6 +281,19 @@ fp8q_status fp8q_permute_pad_quant_noalloc(const void *x, int64_t tokens, int64_
  * status word and returns normally.  No fault, no trap: the context stays usable. */
 fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream);
 
+/* Test hooks for cross-checks against a CPU implementation (no counterpart on the pages).
+ *   fp8q_debug_e4m3_encode_range: out[i] = the E4M3 code (round to nearest even,
+ *     saturating to +-448) that every kernel's fp32 -> E4M3 conversion gives for the fp32
+ *     with bit pattern first_bits + i, i < n (first_bits + n <= 2^32).
+ *   fp8q_debug_exp_spec_range: out[i] = the SwiGLU spec's exp (fp32) of the fp32 with bit
+ *     pattern first_bits + i.
+ *   fp8q_debug_swiglu_spec: y[i] = silu(gate[i]) * up[i] by the SwiGLU spec, fp32 in and
+ *     out (the value fp8q_swiglu_quant quantizes).
+ * Device pointers; float arrays 4-byte aligned.  Errors: ARG, NULL, ALIGN, CUDA. */
+fp8q_status fp8q_debug_e4m3_encode_range(uint32_t first_bits, int64_t n, uint8_t *out, fp8q_stream_t stream);
+fp8q_status fp8q_debug_exp_spec_range(uint32_t first_bits, int64_t n, float *out, fp8q_stream_t stream);
+fp8q_status fp8q_debug_swiglu_spec(const float *gate, const float *up, int64_t n, float *y, fp8q_stream_t stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int fp8q_version(void);
 

@@ -68,6 +68,8 @@ def _declare(L):
         "orc_unpermute_unpad": [V, V, I64, I64, V, V, I64, I32, V],
         "orc_permute_pad_fp8": [V, V, I64, I64, V, I32, I32, I32, V, V, I64, V, V],
         "orc_quantize_rowwise_g": [V, I64, I64, I32, V, V],
+        "orc_e4m3_encode_f32_range": [ctypes.c_uint32, I64, V],
+        "orc_exp_spec_f32_range": [ctypes.c_uint32, I64, V],
         "orc_direct_transpose_g": [V, V, I64, I64, I32, V, V],
     }.items():
         fn = getattr(L, name)
@@ -335,6 +337,20 @@ def unpermute_unpad(y, row_id_map, topk: int, weights=None, y_sf=None):
     rc = lib().orc_unpermute_unpad(_p(yy), _p(sf), rows, H, _p(rmap), _p(w), T, K, _p(out))
     if rc:
         raise OracleError(f"oracle unpermute rejected its arguments (code {rc})")
+    return out
+
+
+def e4m3_encode_f32_range(first: int, n: int) -> np.ndarray:
+    """E4M3 codes of the fp32 values with bit patterns first..first+n-1 (0 for non-finite)."""
+    out = np.empty(n, np.uint8)
+    lib().orc_e4m3_encode_f32_range(first, n, _p(out))
+    return out
+
+
+def exp_spec_f32_range(first: int, n: int) -> np.ndarray:
+    """The SwiGLU spec's exp of the fp32 values with bit patterns first..first+n-1 (0 for NaN)."""
+    out = np.empty(n, np.float32)
+    lib().orc_exp_spec_f32_range(first, n, _p(out))
     return out
 
 

@@ -832,6 +832,34 @@ int orc_unpermute_unpad(const void *y, const uint8_t *y_sf, int64_t rows, int64_
     return 0;
 }
 
+/* Range helpers for the exhaustive cross-checks: inputs are the fp32 values with bit
+ * patterns first .. first + n - 1 (n <= 2^32 - first). */
+void orc_e4m3_encode_f32_range(uint32_t first, int64_t n, uint8_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++) {
+        union {
+            uint32_t u;
+            float f;
+        } v;
+        v.u = first + (uint32_t)i;
+        out[i] = isfinite(v.f) ? orc_e4m3_encode((double)v.f) : 0;
+    }
+}
+
+void orc_exp_spec_f32_range(uint32_t first, int64_t n, float *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++) {
+        union {
+            uint32_t u;
+            float f;
+        } v;
+        v.u = first + (uint32_t)i;
+        out[i] = isnan(v.f) ? 0.0f : orc_exp_spec(v.f);
+    }
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

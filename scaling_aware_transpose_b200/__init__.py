@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
             "fp8q_quantize_rowwise_mx32": ([P, I64, I64, P, P, P], ctypes.c_int),
             "fp8q_direct_transpose_mx32": ([P, P, I64, I64, P, P, P], ctypes.c_int),
             "fp8q_debug_expire_wait": ([ctypes.c_uint64, P], ctypes.c_int),
+            "fp8q_debug_e4m3_encode_range": ([ctypes.c_uint32, I64, P, P], ctypes.c_int),
+            "fp8q_debug_exp_spec_range": ([ctypes.c_uint32, I64, P, P], ctypes.c_int),
+            "fp8q_debug_swiglu_spec": ([P, P, I64, P, P], ctypes.c_int),
             "fp8q_version": ([], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -204,6 +207,19 @@ def fp8q_direct_transpose_mx32(q, sf, rows: int, cols: int, qt, sft, stream=None
 
 def fp8q_debug_expire_wait(timeout_ns: int, stream=None) -> None:
     _check(lib().fp8q_debug_expire_wait(int(timeout_ns), _stream(stream)), "fp8q_debug_expire_wait")
+
+
+def fp8q_debug_e4m3_encode_range(first_bits: int, n: int, out, stream=None) -> None:
+    _check(lib().fp8q_debug_e4m3_encode_range(first_bits, n, _ptr(out), _stream(stream)),
+           "fp8q_debug_e4m3_encode_range")
+
+
+def fp8q_debug_exp_spec_range(first_bits: int, n: int, out, stream=None) -> None:
+    _check(lib().fp8q_debug_exp_spec_range(first_bits, n, _ptr(out), _stream(stream)), "fp8q_debug_exp_spec_range")
+
+
+def fp8q_debug_swiglu_spec(gate, up, n: int, y, stream=None) -> None:
+    _check(lib().fp8q_debug_swiglu_spec(_ptr(gate), _ptr(up), n, _ptr(y), _stream(stream)), "fp8q_debug_swiglu_spec")
 
 
 def fp8q_version() -> int:

@@ -43,6 +43,18 @@ __global__ void expire_wait_kernel(uint64_t timeout_ns, int* status) {
   }
 }
 
+// ---- encoder test hook: the E4M3 conversion every kernel uses, over raw fp32 bit patterns
+__global__ void encode_range_kernel(uint32_t first, int64_t n, uint8_t* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = (uint8_t)cvt_e4m3x2_f32(__uint_as_float(first + (uint32_t)i), 0.0f);
+}
+
+fp8q_status launch_debug_encode_range(uint32_t first, int64_t n, uint8_t* out, cudaStream_t stream) {
+  if (n <= 0) return FP8Q_OK;
+  encode_range_kernel<<<1184, 256, 0, stream>>>(first, n, out);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream) {
   expire_wait_kernel<<<1, 32, 0, stream>>>(timeout_ns, dev.status);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
@@ -110,6 +122,30 @@ const char* fp8q_status_string(fp8q_status s) {
     case FP8Q_ERR_DEVICE: return "a kernel saw invalid data";
   }
   return "unknown status";
+}
+
+fp8q_status fp8q_debug_e4m3_encode_range(uint32_t first_bits, int64_t n, uint8_t* out, fp8q_stream_t stream) {
+  if (n < 0 || n > (int64_t)1 << 32 || (int64_t)first_bits + n > (int64_t)1 << 32) return FP8Q_ERR_ARG;
+  if (n == 0) return FP8Q_OK;
+  if (!out) return FP8Q_ERR_NULL;
+  return fp8q::launch_debug_encode_range(first_bits, n, out, as_stream(stream));
+}
+
+fp8q_status fp8q_debug_exp_spec_range(uint32_t first_bits, int64_t n, float* out, fp8q_stream_t stream) {
+  if (n < 0 || n > (int64_t)1 << 32 || (int64_t)first_bits + n > (int64_t)1 << 32) return FP8Q_ERR_ARG;
+  if (n == 0) return FP8Q_OK;
+  if (!out) return FP8Q_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(out) & 3u) return FP8Q_ERR_ALIGN;
+  return fp8q::launch_debug_exp_spec_range(first_bits, n, out, as_stream(stream));
+}
+
+fp8q_status fp8q_debug_swiglu_spec(const float* gate, const float* up, int64_t n, float* y, fp8q_stream_t stream) {
+  if (n < 0) return FP8Q_ERR_ARG;
+  if (n == 0) return FP8Q_OK;
+  if (!gate || !up || !y) return FP8Q_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(gate) | reinterpret_cast<uintptr_t>(up) | reinterpret_cast<uintptr_t>(y)) & 3u)
+    return FP8Q_ERR_ALIGN;
+  return fp8q::launch_debug_swiglu_spec(gate, up, n, y, as_stream(stream));
 }
 
 int fp8q_version(void) { return 10000; }

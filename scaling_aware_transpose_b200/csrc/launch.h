@@ -61,6 +61,10 @@ fp8q_status launch_quantize_mx32(const void* x, int64_t rows, int64_t cols, uint
 fp8q_status launch_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols, uint8_t* qt,
                                          uint8_t* sft, cudaStream_t stream);
 
+fp8q_status launch_debug_encode_range(uint32_t first, int64_t n, uint8_t* out, cudaStream_t stream);
+fp8q_status launch_debug_exp_spec_range(uint32_t first, int64_t n, float* out, cudaStream_t stream);
+fp8q_status launch_debug_swiglu_spec(const float* g, const float* u, int64_t n, float* y, cudaStream_t stream);
+
 fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace fp8q

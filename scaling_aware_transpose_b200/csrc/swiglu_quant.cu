@@ -166,6 +166,18 @@ __global__ void __launch_bounds__(kThreads, 3) swiglu_quant_kernel(const uint16_
   if (tid < 128) sft[(int64_t)(c0 + tid) * (rows >> 7) + (r0 >> 7)] = (uint8_t)emax;
 }
 
+// Test hooks: the device exp and SwiGLU spec on raw inputs, for cross-checks against the
+// CPU implementation of the same spec.  exp over the fp32 bit patterns first..first+n-1.
+__global__ void exp_spec_range_kernel(uint32_t first, int64_t n, float* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = exp_spec(__uint_as_float(first + (uint32_t)i));
+}
+__global__ void swiglu_spec_kernel(const float* __restrict__ g, const float* __restrict__ u, int64_t n,
+                                   float* __restrict__ y) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = swiglu_spec(g[i], u[i]);
+}
+
 }  // namespace
 
 fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const void* up, int64_t rows, int64_t cols,
@@ -177,6 +189,18 @@ fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const v
   dim3 grid((unsigned)gx, (unsigned)(cols / 128));
   swiglu_quant_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(gate),
                                                      static_cast<const uint16_t*>(up), rows, (int)cols, q, sf, qt, sft);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+fp8q_status launch_debug_exp_spec_range(uint32_t first, int64_t n, float* out, cudaStream_t stream) {
+  if (n <= 0) return FP8Q_OK;
+  exp_spec_range_kernel<<<1184, 256, 0, stream>>>(first, n, out);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+fp8q_status launch_debug_swiglu_spec(const float* g, const float* u, int64_t n, float* y, cudaStream_t stream) {
+  if (n <= 0) return FP8Q_OK;
+  swiglu_spec_kernel<<<1184, 256, 0, stream>>>(g, u, n, y);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

@@ -157,6 +157,16 @@ def test_mx32_host_errors(L):
     assert fd(None, None, 0, 128, None, None, None) == sat.FP8Q_OK
 
 
+def test_debug_hook_host_errors(L):
+    assert L.fp8q_debug_e4m3_encode_range(0xFFFFFFF0, 32, A, None) == sat.FP8Q_ERR_ARG   # past 2^32
+    assert L.fp8q_debug_e4m3_encode_range(0, 16, None, None) == sat.FP8Q_ERR_NULL
+    assert L.fp8q_debug_exp_spec_range(0, 16, A + 2, None) == sat.FP8Q_ERR_ALIGN
+    assert L.fp8q_debug_exp_spec_range(0, -1, A, None) == sat.FP8Q_ERR_ARG
+    assert L.fp8q_debug_swiglu_spec(A, None, 16, A, None) == sat.FP8Q_ERR_NULL
+    assert L.fp8q_debug_swiglu_spec(A, A, 16, A + 1, None) == sat.FP8Q_ERR_ALIGN
+    assert L.fp8q_debug_swiglu_spec(None, None, 0, None, None) == sat.FP8Q_OK
+
+
 def test_permute_host_errors(L):
     f = L.fp8q_permute_pad_quant
 
