@@ -166,9 +166,22 @@ def cpu_baseline(x_bits, budget_s: float = 10.0, max_reps: int = 50):
     rows = x_bits.shape[0]
     step_bytes = BYTES_STEP * rows // ROWS
     avg = sum(times) / len(times)
-    return {"value": round(step_bytes / avg / 1e9, 3), "unit": "GB/s", "cores": oracle.num_threads(),
+    cores = oracle.num_threads()
+    # one thread, on the first 1/8 of the rows (a few seconds)
+    sub = x_bits[: max(128, rows // 8)]
+    oracle.set_num_threads(1)
+    try:
+        t0 = time.perf_counter()
+        q, sf = oracle.quantize_rowwise(sub)
+        oracle.direct_transpose(q, sf)
+        t1 = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": round(step_bytes / avg / 1e9, 3), "unit": "GB/s", "cores": cores,
             "kind": "oracle", "sample": f"{rows}x{COLS} rows of the workload (quantize + direct transpose), "
-                                        f"{reps} repetitions, {sum(times):.1f} s"}
+                                        f"{reps} repetitions, {sum(times):.1f} s",
+            "value_1_thread": round(BYTES_STEP * sub.shape[0] // ROWS / t1 / 1e9, 3),
+            "sample_1_thread": f"{sub.shape[0]}x{COLS} rows, one repetition, {t1:.1f} s"}
 
 
 

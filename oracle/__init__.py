@@ -76,6 +76,7 @@ def _declare(L):
         fn.argtypes, fn.restype = args, ctypes.c_int
     L.orc_exp_spec.argtypes, L.orc_exp_spec.restype = [F], F
     L.orc_num_threads.argtypes, L.orc_num_threads.restype = [], ctypes.c_int
+    L.orc_set_num_threads.argtypes, L.orc_set_num_threads.restype = [ctypes.c_int], None
 
 
 class OracleError(RuntimeError):
@@ -352,6 +353,10 @@ def exp_spec_f32_range(first: int, n: int) -> np.ndarray:
     out = np.empty(n, np.float32)
     lib().orc_exp_spec_f32_range(first, n, _p(out))
     return out
+
+
+def set_num_threads(n: int) -> None:
+    lib().orc_set_num_threads(int(n))
 
 
 def num_threads() -> int:

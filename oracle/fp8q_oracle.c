@@ -868,3 +868,14 @@ int orc_num_threads(void)
     return 1;
 #endif
 }
+
+/* Thread count for the OpenMP loops (the baseline timing at one thread and at all). */
+void orc_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

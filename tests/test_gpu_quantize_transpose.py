@@ -194,3 +194,29 @@ def test_empty_inputs_are_noops():
     qt, sft = sat.direct_transpose(q, sf)
     assert qt.shape == (256, 0)
     device_status_ok()
+
+
+# ------------------------------------------------------------------ 50 random small shapes
+
+def _random_shapes(n=50, seed=123):
+    rng = np.random.default_rng(seed)
+    return [(128 * int(rng.integers(1, 9)), 128 * int(rng.integers(1, 9)), int(rng.integers(0, 1 << 30)))
+            for _ in range(n)]
+
+
+@pytest.mark.parametrize("rows,cols,seed", _random_shapes())
+def test_fifty_random_small_shapes(rows, cols, seed):
+    """T, H in {128..1024} (multiples of 128), seeded; every step of the path (quantize,
+    direct, naive, single pass) against the oracle.  Inputs alternate between the dense
+    and the range-stress recipes."""
+    if seed % 2:
+        x = synthetic.stress(rows=rows, cols=cols, seed=seed % 1000)["x"]
+    else:
+        x = synthetic.scaled_normal(rows, cols, seed=seed % 1000, row_sigma=2.0)
+    check_against_oracle(x, naive=True)
+    q, sf, qt, sft = sat.quantize_rowwise_colwise(dev(x))
+    oq, osf, oqt, osft = oracle.quantize_rowwise_colwise(x)
+    assert_bytes_equal(host(q), oq, "single-pass Q")
+    assert_bytes_equal(host(sf), osf, "single-pass SF")
+    assert_bytes_equal(host(qt), oqt, "single-pass Q^T")
+    assert_bytes_equal(host(sft), osft, "single-pass SF^T")
