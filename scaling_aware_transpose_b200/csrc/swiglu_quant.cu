@@ -32,6 +32,10 @@ constexpr float kC4 = 0x1.555556p-5f, kC5 = 0x1.111112p-7f, kC6 = 0x1.6c16c2p-10
 // rint(t) for |t| < 2^22 is (t + 1.5*2^23) - 1.5*2^23 with both additions rounded to
 // nearest even (the first sum lies in [2^23, 2^24), whose ulp is 1); the integer n is read
 // off the bits of the first sum.  Same result as rintf, without the conversion unit.
+// The spec's two range rules need no select here: after the clamp, a = 89 evaluates to
+// p * 2^128 with p = e^0.277... > 1, which overflows to +inf, and a = -104 to p * 2^-150
+// with p = e^-0.027... < 1, which rounds to +0 - exactly the values the rules assign to
+// a > 89 and a < -104 (checked on every fp32 input against the CPU spec).
 __device__ __forceinline__ float exp_spec(float a) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   const float ac = fminf(fmaxf(a, -104.0f), 89.0f);  // keeps n in [-150, 128]
@@ -50,8 +54,7 @@ __device__ __forceinline__ float exp_spec(float a) {
   const int ni = __float_as_int(tm) - 0x4B400000;
   const int n1 = ni >> 1;  // floor(n / 2)
   const int n2 = ni - n1;
-  const float res = __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
-  return a > 89.0f ? __int_as_float(0x7F800000) : (a < -104.0f ? 0.0f : res);
+  return __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
 }
 
 __device__ __forceinline__ float swiglu_spec(float g, float u) {
@@ -101,16 +104,16 @@ __global__ void __launch_bounds__(kThreads, 3) swiglu_quant_kernel(const uint16_
     float y[16];
     const uint32_t gw[8] = {gv[p][0].x, gv[p][0].y, gv[p][0].z, gv[p][0].w, gv[p][1].x, gv[p][1].y, gv[p][1].z, gv[p][1].w};
     const uint32_t uw[8] = {uv[p][0].x, uv[p][0].y, uv[p][0].z, uv[p][0].w, uv[p][1].x, uv[p][1].y, uv[p][1].z, uv[p][1].w};
-    uint32_t amax = 0u;
+    float amax = 0.0f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       y[2 * k] = swiglu_spec(__uint_as_float(gw[k] << 16), __uint_as_float(uw[k] << 16));
       y[2 * k + 1] = swiglu_spec(__uint_as_float(gw[k] & 0xFFFF0000u), __uint_as_float(uw[k] & 0xFFFF0000u));
-      amax = max(amax, max(__float_as_uint(y[2 * k]) & 0x7FFFFFFFu, __float_as_uint(y[2 * k + 1]) & 0x7FFFFFFFu));
+      amax = fmaxf(amax, fmaxf(fabsf(y[2 * k]), fabsf(y[2 * k + 1])));  // finite y: plain magnitude max
     }
 #pragma unroll
-    for (int o = 4; o >= 1; o >>= 1) amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    const int e = tile_exponent(__uint_as_float(amax));
+    for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    const int e = tile_exponent(amax);
     const float s = exp2_neg(e);
     uint4 codes;
     codes.x = cvt_e4m3x2_f32(y[0] * s, y[1] * s) | (cvt_e4m3x2_f32(y[2] * s, y[3] * s) << 16);
