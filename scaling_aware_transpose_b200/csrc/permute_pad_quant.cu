@@ -9,8 +9,8 @@
 // byte 127) to a multiple of `align`.
 //
 // Launches: (1) per-chunk expert histograms, (2) one CTA scans them into padded expert
-// offsets and per-chunk bases, (3) one warp per chunk assigns stable ranks with
-// __match_any_sync, (4) the streaming scatter-quantize over all (token, tile) pairs, whose
+// offsets and per-chunk bases, (3) stable ranks within each chunk with __match_any_sync
+// (eight warps per chunk for up to 512 experts, one warp beyond), (4) the streaming scatter-quantize over all (token, tile) pairs, whose
 // trailing CTAs zero-fill the padding rows.  Workspace: counts[C][E], bases[C][E], totals[E].
 // The FP8-input variant (the dispatch already delivered row-wise codes and scales) shares
 // (1)-(3) and the padding; its step (4) copies each token's codes and scale bytes to its
@@ -46,67 +46,90 @@ __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ 
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
-// Inclusive warp scan of v.
-__device__ __forceinline__ int64_t warp_incl_scan(int64_t v, int lane) {
+// Inclusive warp scan of a 32-bit value.
+__device__ __forceinline__ int32_t warp_incl_scan32(int32_t v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int64_t t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    const int32_t t = __shfl_up_sync(0xFFFFFFFFu, v, o);
     if (lane >= o) v += t;
   }
   return v;
 }
 
-// One CTA of 1024 threads (32 warps):
-//  (1) warp w sums expert e's counts over the chunks (e = w, w + 32, ...) -> totals[e];
-//  (2) block-wide exclusive scan of the padded sizes ceil(total/align)*align -> offsets;
-//  (3) warp per expert again: exclusive scan over the chunks -> bases[c][e].
+// One CTA of 1024 threads (32 warps); totals and offsets stay in shared memory, so the
+// kernel is a short chain: (1) warp w sums expert e's counts over the chunks (e = w,
+// w + 32, ...; eight loads in flight per lane) -> totals; (2) exclusive scan of the padded
+// sizes ceil(total/align)*align over the experts (per-thread runs, a warp scan and a scan
+// of the 32 warp sums) -> offsets; (3) warp per expert again: exclusive scan over the
+// chunks -> bases[c][e].  Every value fits in int32: the host caps the padded row count
+// below 2^31.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int64_t C, int E, int align,
                                                     int32_t* __restrict__ offsets, int32_t* __restrict__ bases,
                                                     int32_t* __restrict__ totals) {
-  __shared__ int64_t part[1024];
+  __shared__ int32_t s_tot[kMaxExperts];
+  __shared__ int32_t s_off[kMaxExperts];
+  __shared__ int32_t s_warp[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = warp; e < E; e += 32) {
-    int64_t acc = 0;
-    for (int64_t c = lane; c < C; c += 32) acc += counts[c * E + e];
+    int32_t acc = 0;
+    for (int64_t c0 = 0; c0 < C; c0 += 8 * 32) {
+      int32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + u * 32 + lane;
+        v[u] = c < C ? __ldg(counts + c * E + e) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc += v[u];
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if (lane == 0) totals[e] = (int32_t)acc;
+    if (lane == 0) {
+      s_tot[e] = acc;
+      totals[e] = acc;
+    }
   }
   __syncthreads();
-  // thread tid owns experts [tid*per, (tid+1)*per)
-  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;  // experts per thread
   const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-  int64_t local = 0;
-  for (int e = e0; e < e1; ++e) local += ((int64_t)totals[e] + align - 1) / align * align;
-  part[tid] = local;
+  int32_t local = 0;
+  for (int e = e0; e < e1; ++e) local += (s_tot[e] + align - 1) / align * align;
+  const int32_t incl = warp_incl_scan32(local, lane);
+  if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
-  for (int o = 1; o < (int)blockDim.x; o <<= 1) {  // inclusive scan (Hillis-Steele)
-    const int64_t v = tid >= o ? part[tid - o] : 0;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
+  if (warp == 0) {
+    const int32_t w = s_warp[lane];
+    s_warp[lane] = warp_incl_scan32(w, lane) - w;  // exclusive prefix of the warp sums
   }
-  int64_t run = part[tid] - local;
+  __syncthreads();
+  int32_t run = s_warp[warp] + incl - local;
   for (int e = e0; e < e1; ++e) {
-    offsets[e] = (int32_t)run;
-    run += ((int64_t)totals[e] + align - 1) / align * align;
+    s_off[e] = run;
+    offsets[e] = run;
+    run += (s_tot[e] + align - 1) / align * align;
   }
-  if (tid == blockDim.x - 1) offsets[E] = (int32_t)part[tid];
+  if (tid == (int)blockDim.x - 1) offsets[E] = run;  // threads past the last expert hold the total
   __syncthreads();
   for (int e = warp; e < E; e += 32) {
-    int64_t carry = offsets[e];
-    for (int64_t c0 = 0; c0 < C; c0 += 32) {
-      const int64_t c = c0 + lane;
-      const int64_t v = c < C ? counts[c * E + e] : 0;
-      const int64_t incl = warp_incl_scan(v, lane);
-      if (c < C) bases[c * E + e] = (int32_t)(carry + incl - v);
-      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    int32_t carry = s_off[e];
+    for (int64_t c0 = 0; c0 < C; c0 += 8 * 32) {
+      int32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + u * 32 + lane;
+        v[u] = c < C ? __ldg(counts + c * E + e) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + u * 32 + lane;
+        const int32_t inc = warp_incl_scan32(v[u], lane);
+        if (c < C) bases[c * E + e] = carry + inc - v[u];
+        carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+      }
     }
   }
 }
 
-// One warp per chunk: stable destination rows in (t, s) order.  The chunk's routing ids
-// are loaded up front so that the 32 ranking steps do not wait on memory.
 __global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
                                                   const int32_t* __restrict__ bases, int32_t* __restrict__ row_id_map) {
   extern __shared__ int32_t run[];
@@ -134,6 +157,69 @@ __global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ id
     if (ok) {
       row_id_map[p] = base + rank;
       if (rank == 0) run[e] = base + __popc(same);
+    } else if (live) {
+      row_id_map[p] = -1;
+    }
+    __syncwarp();
+  }
+}
+
+// Rank with 8 warps per chunk, for E <= kRankMultiMaxE (per-warp counts in shared
+// memory): warp w owns pairs 128w..128w+127 of the chunk.  (A) each warp counts its pairs
+// per expert; (B) per expert, an exclusive prefix over the warps on top of the chunk's
+// base; (C) each warp ranks its pairs from its own bases.  Same stable (t, s) order as
+// rank_kernel with 8 serial steps per warp instead of 32.
+constexpr int kRankWarps = 8;
+constexpr int kRankMultiMaxE = 512;
+__global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32_t* __restrict__ idx, int64_t npairs,
+                                                                     int E, const int32_t* __restrict__ bases,
+                                                                     int32_t* __restrict__ row_id_map) {
+  extern __shared__ int32_t s_cnt[];  // [kRankWarps][E]
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  constexpr int kPer = kChunk / kRankWarps / 32;  // iterations per warp
+  const int64_t p0 = (int64_t)blockIdx.x * kChunk + w * (kChunk / kRankWarps);
+  int32_t ids[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    ids[i] = p < npairs ? __ldg(idx + p) : -1;
+  }
+  for (int e = tid; e < kRankWarps * E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  int32_t* mine = s_cnt + w * E;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    const int32_t e = ids[i];
+    const bool ok = p < npairs && e >= 0 && e < E;
+    const unsigned same = __match_any_sync(0xFFFFFFFFu, ok ? e : -1 - lane);
+    if (ok && lane == __ffs(same) - 1) mine[e] += __popc(same);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int32_t run = bases[(int64_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int ww = 0; ww < kRankWarps; ++ww) {
+      const int32_t v = s_cnt[ww * E + e];
+      s_cnt[ww * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    const bool live = p < npairs;
+    const int32_t e = ids[i];
+    const bool ok = live && e >= 0 && e < E;
+    const unsigned same = __match_any_sync(0xFFFFFFFFu, ok ? e : -1 - lane);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    const int base = ok ? mine[e] : 0;
+    __syncwarp();
+    if (ok) {
+      row_id_map[p] = base + rank;
+      if (lane == __ffs(same) - 1) mine[e] = base + __popc(same);
     } else if (live) {
       row_id_map[p] = -1;
     }
@@ -301,7 +387,11 @@ fp8q_status route(const DeviceInfo& dev, int64_t tokens, const int32_t* topk_idx
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   scan_kernel<<<1, 1024, 0, stream>>>(counts, C, E, align, expert_offsets, bases, totals);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  rank_kernel<<<(unsigned)C, 32, hist_smem, stream>>>(topk_idx, npairs, E, bases, row_id_map);
+  if (E <= kRankMultiMaxE)
+    rank_multi_kernel<<<(unsigned)C, kRankWarps * 32, (size_t)kRankWarps * E * sizeof(int32_t), stream>>>(
+        topk_idx, npairs, E, bases, row_id_map);
+  else
+    rank_kernel<<<(unsigned)C, 32, hist_smem, stream>>>(topk_idx, npairs, E, bases, row_id_map);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

@@ -183,3 +183,14 @@ def test_permute_fp8_bad_index_sets_device_status():
     idx = torch.tensor([[0], [1], [9], [2]], dtype=torch.int32, device="cuda")
     sat.permute_pad_fp8(q, sf, idx, 4, 16)
     assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE
+
+
+@pytest.mark.parametrize("tokens,E,K", [(700, 300, 4), (2500, 512, 2), (1800, 513, 3), (600, 4096, 8)])
+def test_permute_many_experts(tokens, E, K):
+    """Routing with many experts: the eight-warp rank path up to 512 experts, the one-warp
+    path beyond (513 and the 4096 maximum), uniform routing so most experts are hit."""
+    rng = np.random.default_rng(E)
+    idx = np.argsort(rng.random((tokens, E)), axis=1)[:, :K].astype(np.int32)
+    d = {"x": synthetic.scaled_normal(tokens, 128, seed=E), "topk_idx": np.ascontiguousarray(idx)}
+    check_permute(d, E, 16)
+    check_permute_fp8(d["x"], d["topk_idx"], E, 16)
