@@ -71,8 +71,7 @@ __global__ void __launch_bounds__(kThreads, kGrouped ? 6 : 8) direct_transpose_k
   __syncthreads();
   const uint32_t ew = reinterpret_cast<const uint32_t*>(e_row)[tid & 31];
   int m = (int)max(max(ew & 0xFFu, (ew >> 8) & 0xFFu), max((ew >> 16) & 0xFFu, ew >> 24));
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+  m = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)m);
   const int emax = m;
   // ---- 2. shift and stage
 #pragma unroll

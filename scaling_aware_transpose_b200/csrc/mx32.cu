@@ -15,9 +15,9 @@
 //
 // direct_transpose_mx32_kernel: the 128x128 block-per-CTA direct transpose with 16 MX
 // blocks per CTA tile.  Each row's four scale bytes (one per 32-column group) move as one
-// 32-bit word; every warp reduces the packed Smax words of all four row groups itself
-// (a byte-wise max, __vmaxu4, over five shuffles each, the four chains interleaved), so
-// one barrier suffices as in the 128 kernel.  The shift of a 16-byte row chunk uses its
+// 32-bit word; every warp computes the Smax of all sixteen (row group, column group)
+// blocks itself with single-instruction warp max reductions (__reduce_max_sync), so one
+// barrier suffices as in the 128 kernel.  The shift of a 16-byte row chunk uses its
 // own 32x32 block's k; staging and the byte transpose (8 tokens x 8 channels per lane)
 // are those of the 128 kernel.
 #include "common.cuh"
@@ -72,12 +72,6 @@ constexpr int kPasses = 4;
 
 __device__ __forceinline__ int chunk_pos(int r, int c) { return c ^ ((r >> 3) & 7); }
 __device__ __forceinline__ int byte_of(uint32_t w, int i) { return (int)((w >> (8 * i)) & 0xFFu); }
-// Byte c of each of four words, packed (word i -> byte i).
-__device__ __forceinline__ uint32_t gather_byte4(const uint32_t (&w)[4], int c) {
-  const uint32_t lo = __byte_perm(w[0], w[1], (uint32_t)(c | ((c + 4) << 4)));
-  const uint32_t hi = __byte_perm(w[2], w[3], (uint32_t)(c | ((c + 4) << 4)));
-  return __byte_perm(lo, hi, 0x5410);
-}
 
 __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(const uint8_t* __restrict__ q,
                                                                           const uint8_t* __restrict__ sf, int64_t rows,
@@ -100,18 +94,22 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   // the row's 4 scale bytes: 4-byte aligned (rows of cols/32 bytes, cols % 128 == 0)
   if (tid < 128) e_row[tid] = __ldg(reinterpret_cast<const uint32_t*>(sf + (r0 + tid) * ngr + (c0 >> 5)));
   __syncthreads();
-  uint32_t e_max[4];  // per row group: packed Smax bytes of column groups 0..3
+  // Smax of every (row group, column group) with single-instruction warp reductions; keep
+  // the two packed words this thread needs: its own column group over the row groups,
+  // and the SF^T channel's column group over the row groups.
+  const int cg = sub >> 1;            // 32-column group of this thread's 16-byte chunks
+  const int cg_t = (tid >> 5) & 3;    // column group of channel c0 + tid (SF^T word)
+  uint32_t smax_mine = 0, smax_sft = 0;
 #pragma unroll
-  for (int rg = 0; rg < 4; ++rg) e_max[rg] = e_row[32 * rg + (tid & 31)];
+  for (int rg = 0; rg < 4; ++rg) {
+    const uint32_t w = e_row[32 * rg + (tid & 31)];
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1)
-#pragma unroll
-    for (int rg = 0; rg < 4; ++rg) e_max[rg] = __vmaxu4(e_max[rg], __shfl_xor_sync(0xFFFFFFFFu, e_max[rg], o));
-  // byte i of smax_mine: Smax of (row group i, this thread's column group); of smax_sft:
-  // Smax of (row group i, column group of channel c0 + tid) for the SF^T word
-  const int cg = sub >> 1;  // 32-column group of this thread's 16-byte chunks
-  const uint32_t smax_mine = gather_byte4(e_max, cg);
-  const uint32_t smax_sft = gather_byte4(e_max, (tid >> 5) & 3);
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, (w >> (8 * c)) & 0xFFu);
+      smax_mine |= (c == cg ? m : 0u) << (8 * rg);
+      smax_sft |= (c == cg_t ? m : 0u) << (8 * rg);
+    }
+  }
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
     const int rl = p * 32 + rsub;  // row group p

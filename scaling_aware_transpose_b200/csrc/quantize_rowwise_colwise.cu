@@ -89,8 +89,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     __syncthreads();
     const uint32_t w = reinterpret_cast<const uint32_t*>(e_row)[tid & 31];
     int m = (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24));
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    m = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)m);
     emax = m - 127;
   }
 

@@ -136,8 +136,7 @@ __global__ void __launch_bounds__(kThreads, 3) swiglu_quant_kernel(const uint16_
   if (tid < 32) {
     const uint32_t w = reinterpret_cast<const uint32_t*>(e_row)[tid];
     int m = (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24));
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    m = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)m);
     if (tid == 0) e_max_sh = m;
   }
   __syncthreads();
