@@ -66,7 +66,7 @@ namespace {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(fp8q_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
-constexpr int64_t kMaxDim = 0x7FFFFFFFll;  // TMA coordinates and group offsets are int32
+constexpr int64_t kMaxDim = 0x7FFFFFFFll;  // grid sizes, group offsets and row ids are int32
 
 // Shape rules shared by the two transposes.
 fp8q_status check_transpose_args(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols,
