@@ -134,3 +134,15 @@ CONFIGS = {
     "swiglu": swiglu,
     "stress": stress,
 }
+
+
+def device_normal(rows: int, cols: int, seed: int, device, row_sigma: float = 1.0):
+    """Large inputs made on the device (too big to draw on the host in a test): a seeded
+    torch generator gives z ~ N(0,1) times a lognormal(0, row_sigma) factor per row, as
+    BF16.  Both sides use the same bytes: the GPU reads the tensor, the oracle its rows
+    copied back."""
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    z = torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32)
+    f = torch.exp(row_sigma * torch.randn((rows, 1), generator=g, device=device, dtype=torch.float32))
+    return (z * f).to(torch.bfloat16)
