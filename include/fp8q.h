@@ -289,10 +289,15 @@ fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream);
  *     pattern first_bits + i.
  *   fp8q_debug_swiglu_spec: y[i] = silu(gate[i]) * up[i] by the SwiGLU spec, fp32 in and
  *     out (the value fp8q_swiglu_quant quantizes).
+ *   fp8q_debug_silu_bf16: y[i] = silu(gate[i]) for n BF16 gate values (n even, gate
+ *     4-byte and y 8-byte aligned), computed the way fp8q_swiglu_quant computes it (the
+ *     spec's values tabulated in shared memory, looked up, closed forms outside the
+ *     table's range).
  * Device pointers; float arrays 4-byte aligned.  Errors: ARG, NULL, ALIGN, CUDA. */
 fp8q_status fp8q_debug_e4m3_encode_range(uint32_t first_bits, int64_t n, uint8_t *out, fp8q_stream_t stream);
 fp8q_status fp8q_debug_exp_spec_range(uint32_t first_bits, int64_t n, float *out, fp8q_stream_t stream);
 fp8q_status fp8q_debug_swiglu_spec(const float *gate, const float *up, int64_t n, float *y, fp8q_stream_t stream);
+fp8q_status fp8q_debug_silu_bf16(const void *gate, int64_t n, float *y, fp8q_stream_t stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int fp8q_version(void);

@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "fp8q_debug_e4m3_encode_range": ([ctypes.c_uint32, I64, P, P], ctypes.c_int),
             "fp8q_debug_exp_spec_range": ([ctypes.c_uint32, I64, P, P], ctypes.c_int),
             "fp8q_debug_swiglu_spec": ([P, P, I64, P, P], ctypes.c_int),
+            "fp8q_debug_silu_bf16": ([P, I64, P, P], ctypes.c_int),
             "fp8q_version": ([], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -220,6 +221,10 @@ def fp8q_debug_exp_spec_range(first_bits: int, n: int, out, stream=None) -> None
 
 def fp8q_debug_swiglu_spec(gate, up, n: int, y, stream=None) -> None:
     _check(lib().fp8q_debug_swiglu_spec(_ptr(gate), _ptr(up), n, _ptr(y), _stream(stream)), "fp8q_debug_swiglu_spec")
+
+
+def fp8q_debug_silu_bf16(gate, n: int, y, stream=None) -> None:
+    _check(lib().fp8q_debug_silu_bf16(_ptr(gate), n, _ptr(y), _stream(stream)), "fp8q_debug_silu_bf16")
 
 
 def fp8q_version() -> int:

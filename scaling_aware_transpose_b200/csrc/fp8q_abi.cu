@@ -148,6 +148,14 @@ fp8q_status fp8q_debug_swiglu_spec(const float* gate, const float* up, int64_t n
   return fp8q::launch_debug_swiglu_spec(gate, up, n, y, as_stream(stream));
 }
 
+fp8q_status fp8q_debug_silu_bf16(const void* gate, int64_t n, float* y, fp8q_stream_t stream) {
+  if (n < 0 || n % 2) return FP8Q_ERR_ARG;
+  if (n == 0) return FP8Q_OK;
+  if (!gate || !y) return FP8Q_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(gate) & 3u) || (reinterpret_cast<uintptr_t>(y) & 7u)) return FP8Q_ERR_ALIGN;
+  return fp8q::launch_debug_silu_bf16(gate, n, y, as_stream(stream));
+}
+
 int fp8q_version(void) { return 10000; }
 
 fp8q_status fp8q_last_device_status(fp8q_stream_t stream) {

@@ -64,6 +64,7 @@ fp8q_status launch_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, in
 fp8q_status launch_debug_encode_range(uint32_t first, int64_t n, uint8_t* out, cudaStream_t stream);
 fp8q_status launch_debug_exp_spec_range(uint32_t first, int64_t n, float* out, cudaStream_t stream);
 fp8q_status launch_debug_swiglu_spec(const float* g, const float* u, int64_t n, float* y, cudaStream_t stream);
+fp8q_status launch_debug_silu_bf16(const void* g, int64_t n, float* y, cudaStream_t stream);
 
 fp8q_status launch_debug_expire_wait(const DeviceInfo& dev, uint64_t timeout_ns, cudaStream_t stream);
 

@@ -17,6 +17,26 @@
 //   silu(g) = g / (1 + exp(-g));   y = silu(g) * u.
 // Constants (each derived from its definition): L2E = fp32(log2 e); LN2_HI = ln 2 cut
 // to the top 15 mantissa bits; LN2_LO = fp32(ln 2 - LN2_HI); 1/k! rounded to fp32.
+//
+// silu(g) depends on g alone and g is BF16, so it takes at most 65536 values.  Outside
+// one magnitude range the spec reduces to a single IEEE operation (each fact checked on
+// every BF16 input against the CPU spec):
+//   |g| < BF16 0x33C1 (about 9e-8): 1 + exp(-g) rounds to exactly 2, silu(g) = RN(g * 0.5);
+//   g >= 89:  exp(-g) <= 2^-24, 1 + exp(-g) rounds to 1, silu(g) = g (true from 16.75 on);
+//   g <= -89: exp(-g) = +inf (the exp clamp), silu(g) = g / inf = -0;
+// the last two together are max(g, -0).  The 2 x 3825 values in between are computed by
+// the spec itself into a shared-memory table at the start of each CTA, and the element
+// loop looks them up: both BF16 values of a word at once (their magnitudes clamped into
+// the range with 16-bit-lane min/max, the sign picking the half of the table), with a
+// warp vote sending the rare warp that saw an input outside the range through the
+// closed forms.  The CTAs are persistent (two per SM), so the table costs a few
+// microseconds per launch while the lookup replaces ~40 instructions per element (the
+// exp, the IEEE divide); every value is still the spec's, bit for bit.
+//
+// Block loop: CTA i takes blocks i, i + gridDim.x, ... (column blocks fastest).  Each
+// thread holds its 4 passes of gate/up in registers and refills a pass with the next
+// block's data as soon as it has consumed it, so three passes of loads are in flight
+// while it computes.
 #include "common.cuh"
 #include "launch.h"
 
@@ -57,115 +77,201 @@ __device__ __forceinline__ float exp_spec(float a) {
   return __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
 }
 
-__device__ __forceinline__ float swiglu_spec(float g, float u) {
-  const float den = __fadd_rn(1.0f, exp_spec(-g));
-  return __fmul_rn(__fdiv_rn(g, den), u);
+__device__ __forceinline__ float silu_spec(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, exp_spec(-g))); }
+__device__ __forceinline__ float swiglu_spec(float g, float u) { return __fmul_rn(silu_spec(g), u); }
+
+// The silu table: BF16 magnitudes kSiluLo..kSiluHi-1, positive g at 0..kTabN-1, negative g
+// at kNegBase..kNegBase+kTabN-1 (entries between are unused).
+constexpr uint32_t kSiluLo = 0x33C1u;
+constexpr uint32_t kSiluHi = 0x42B2u;  // 89
+constexpr uint32_t kTabN = kSiluHi - kSiluLo;
+constexpr uint32_t kNegBase = 4096;
+constexpr int kTab = (int)(kNegBase + kTabN);
+
+__device__ __forceinline__ void build_silu_table(float* tab) {
+  for (int i = threadIdx.x; i < kTab; i += blockDim.x) {
+    const uint32_t ui = (uint32_t)i;
+    if (ui >= kTabN && ui < kNegBase) continue;  // unused gap
+    const uint32_t h = ui < kTabN ? kSiluLo + ui : 0x8000u | (kSiluLo + ui - kNegBase);
+    tab[i] = silu_spec(__uint_as_float(h << 16));
+  }
+}
+
+__device__ __forceinline__ uint32_t umin16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float sel_f32(bool p, float a, float b) {
+  float r;
+  asm("{.reg .pred q; setp.ne.u32 q, %1, 0; selp.f32 %0, %2, %3, q;}" : "=f"(r) : "r"((uint32_t)p), "f"(a), "f"(b));
+  return r;
+}
+
+// Both BF16 values of a word at once: magnitudes clamped into the table's range (16-bit
+// lanes), the sign adding 4096 to the index.  acc collects any clamped-away bits.
+__device__ __forceinline__ void silu_lookup2(const float* tab, uint32_t w, float& lo, float& hi, uint32_t& acc) {
+  const uint32_t m2 = w & 0x7FFF7FFFu;
+  const uint32_t c2 = umin16x2(umax16x2(m2, kSiluLo * 0x10001u), (kSiluHi - 1) * 0x10001u);
+  acc |= m2 ^ c2;
+  const uint32_t key2 = c2 + ((w >> 3) & 0x10001000u);
+  lo = tab[(key2 & 0xFFFFu) - kSiluLo];
+  hi = tab[(key2 >> 16) - kSiluLo];
+}
+
+__device__ __forceinline__ float silu_fix(float v, uint32_t h, float g) {
+  const uint32_t d = (h & 0x7FFFu) - kSiluLo;  // wraps to >= 2^31 below the range
+  const float out = sel_f32((int)d < 0, __fmul_rn(g, 0.5f), fmaxf(g, -0.0f));
+  return sel_f32(d < kTabN, v, out);
 }
 
 constexpr int kThreads = 256;
 constexpr int kPasses = 4;  // 4 passes x 32 rows x (8 threads x 16 elements)
+constexpr int kMinBlocks = 2;
 
 __device__ __forceinline__ uint32_t swizzled_chunk(int row, int chunk) { return (uint32_t)(chunk ^ ((row >> 2) & 7)); }
 
-__global__ void __launch_bounds__(kThreads, 3) swiglu_quant_kernel(const uint16_t* __restrict__ gate,
-                                                                const uint16_t* __restrict__ up, int64_t rows, int cols,
-                                                                uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
-                                                                uint8_t* __restrict__ qt, uint8_t* __restrict__ sft) {
+struct BlockIn {
+  uint4 g[kPasses][2], u[kPasses][2];
+};
+
+// gate/up of pass p (rows p*32 + rsub) of one 128x128 block: 16 elements per thread.
+__device__ __forceinline__ void load_pass(BlockIn& in, int p, const uint16_t* __restrict__ gate,
+                                          const uint16_t* __restrict__ up, int64_t rows, int cols, int64_t r0, int c0,
+                                          int rsub, int sub) {
+  const int64_t r = r0 + p * 32 + rsub;
+  if (r < rows) {
+    const int64_t base = r * cols + c0 + sub * 16;
+    in.g[p][0] = ld_stream(reinterpret_cast<const uint4*>(gate + base));
+    in.g[p][1] = ld_stream(reinterpret_cast<const uint4*>(gate + base + 8));
+    in.u[p][0] = ld_stream(reinterpret_cast<const uint4*>(up + base));
+    in.u[p][1] = ld_stream(reinterpret_cast<const uint4*>(up + base + 8));
+  } else {
+    in.g[p][0] = in.g[p][1] = in.u[p][0] = in.u[p][1] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(const uint16_t* __restrict__ gate,
+                                                                         const uint16_t* __restrict__ up, int64_t rows,
+                                                                         int cols, int nblk,
+                                                                         uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                                                                         uint8_t* __restrict__ qt,
+                                                                         uint8_t* __restrict__ sft) {
+  __shared__ float silu_tab[kTab];
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
   __shared__ int e_max_sh;
   const int tid = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.x * 128;  // row block (grid.x has the larger range)
-  const int c0 = blockIdx.y * 128;
   const int ncb = cols >> 7;
   const int sub = tid & 7;      // 16-element chunk of the row tile
   const int rsub = tid >> 3;    // row within a pass (0..31)
 
-  // ---- load gate/up for all passes first (memory-level parallelism)
-  uint4 gv[kPasses][2], uv[kPasses][2];
+  int blk = blockIdx.x;
+  BlockIn in;
 #pragma unroll
-  for (int p = 0; p < kPasses; ++p) {
-    const int64_t r = r0 + p * 32 + rsub;
-    if (r < rows) {
-      const int64_t base = r * cols + c0 + sub * 16;
-      gv[p][0] = ld_stream(reinterpret_cast<const uint4*>(gate + base));
-      gv[p][1] = ld_stream(reinterpret_cast<const uint4*>(gate + base + 8));
-      uv[p][0] = ld_stream(reinterpret_cast<const uint4*>(up + base));
-      uv[p][1] = ld_stream(reinterpret_cast<const uint4*>(up + base + 8));
-    } else {
-      gv[p][0] = gv[p][1] = uv[p][0] = uv[p][1] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  // ---- y, row-wise quantization
+  for (int p = 0; p < kPasses; ++p)
+    load_pass(in, p, gate, up, rows, cols, (int64_t)(blk / ncb) * 128, (blk % ncb) * 128, rsub, sub);
+  build_silu_table(silu_tab);
+  __syncthreads();
+  for (;;) {
+    const int64_t r0 = (int64_t)(blk / ncb) * 128;
+    const int c0 = (blk % ncb) * 128;
+    const int next = blk + (int)gridDim.x;
+    const int64_t nr0 = (int64_t)(next / ncb) * 128;
+    const int nc0 = (next % ncb) * 128;
+    // ---- y, row-wise quantization
 #pragma unroll
-  for (int p = 0; p < kPasses; ++p) {
-    const int rl = p * 32 + rsub;
-    const int64_t r = r0 + rl;
-    float y[16];
-    const uint32_t gw[8] = {gv[p][0].x, gv[p][0].y, gv[p][0].z, gv[p][0].w, gv[p][1].x, gv[p][1].y, gv[p][1].z, gv[p][1].w};
-    const uint32_t uw[8] = {uv[p][0].x, uv[p][0].y, uv[p][0].z, uv[p][0].w, uv[p][1].x, uv[p][1].y, uv[p][1].z, uv[p][1].w};
-    float amax = 0.0f;
+    for (int p = 0; p < kPasses; ++p) {
+      const int rl = p * 32 + rsub;
+      const int64_t r = r0 + rl;
+      float y[16];
+      const uint32_t gw[8] = {in.g[p][0].x, in.g[p][0].y, in.g[p][0].z, in.g[p][0].w,
+                              in.g[p][1].x, in.g[p][1].y, in.g[p][1].z, in.g[p][1].w};
+      const uint32_t uw[8] = {in.u[p][0].x, in.u[p][0].y, in.u[p][0].z, in.u[p][0].w,
+                              in.u[p][1].x, in.u[p][1].y, in.u[p][1].z, in.u[p][1].w};
+      uint32_t acc = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      y[2 * k] = swiglu_spec(__uint_as_float(gw[k] << 16), __uint_as_float(uw[k] << 16));
-      y[2 * k + 1] = swiglu_spec(__uint_as_float(gw[k] & 0xFFFF0000u), __uint_as_float(uw[k] & 0xFFFF0000u));
-      amax = fmaxf(amax, fmaxf(fabsf(y[2 * k]), fabsf(y[2 * k + 1])));  // finite y: plain magnitude max
-    }
+      for (int k = 0; k < 8; ++k) silu_lookup2(silu_tab, gw[k], y[2 * k], y[2 * k + 1], acc);
+      if (__any_sync(0xFFFFFFFFu, acc != 0u)) {  // an input outside the table in this warp
 #pragma unroll
-    for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    const int e = tile_exponent(amax);
-    const float s = exp2_neg(e);
-    uint4 codes;
-    codes.x = cvt_e4m3x2_f32(y[0] * s, y[1] * s) | (cvt_e4m3x2_f32(y[2] * s, y[3] * s) << 16);
-    codes.y = cvt_e4m3x2_f32(y[4] * s, y[5] * s) | (cvt_e4m3x2_f32(y[6] * s, y[7] * s) << 16);
-    codes.z = cvt_e4m3x2_f32(y[8] * s, y[9] * s) | (cvt_e4m3x2_f32(y[10] * s, y[11] * s) << 16);
-    codes.w = cvt_e4m3x2_f32(y[12] * s, y[13] * s) | (cvt_e4m3x2_f32(y[14] * s, y[15] * s) << 16);
-    if (r < rows) {
-      *reinterpret_cast<uint4*>(q + r * cols + c0 + sub * 16) = codes;
-      if (sub == 0) sf[r * ncb + (c0 >> 7)] = (uint8_t)(e + 127);
+        for (int k = 0; k < 8; ++k) {
+          y[2 * k] = silu_fix(y[2 * k], gw[k] & 0xFFFFu, __uint_as_float(gw[k] << 16));
+          y[2 * k + 1] = silu_fix(y[2 * k + 1], gw[k] >> 16, __uint_as_float(gw[k] & 0xFFFF0000u));
+        }
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        y[2 * k] = __fmul_rn(y[2 * k], __uint_as_float(uw[k] << 16));
+        y[2 * k + 1] = __fmul_rn(y[2 * k + 1], __uint_as_float(uw[k] & 0xFFFF0000u));
+        amax = fmaxf(amax, fmaxf(fabsf(y[2 * k]), fabsf(y[2 * k + 1])));  // finite y: plain magnitude max
+      }
+#pragma unroll
+      for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      const int e = tile_exponent(amax);
+      const float s = exp2_neg(e);
+      uint4 codes;
+      codes.x = cvt_e4m3x2_f32(y[0] * s, y[1] * s) | (cvt_e4m3x2_f32(y[2] * s, y[3] * s) << 16);
+      codes.y = cvt_e4m3x2_f32(y[4] * s, y[5] * s) | (cvt_e4m3x2_f32(y[6] * s, y[7] * s) << 16);
+      codes.z = cvt_e4m3x2_f32(y[8] * s, y[9] * s) | (cvt_e4m3x2_f32(y[10] * s, y[11] * s) << 16);
+      codes.w = cvt_e4m3x2_f32(y[12] * s, y[13] * s) | (cvt_e4m3x2_f32(y[14] * s, y[15] * s) << 16);
+      if (r < rows) {
+        *reinterpret_cast<uint4*>(q + r * cols + c0 + sub * 16) = codes;
+        if (sub == 0) sf[r * ncb + (c0 >> 7)] = (uint8_t)(e + 127);
+      }
+      if (qt != nullptr) {
+        *reinterpret_cast<uint4*>(tile + rl * 128 + (swizzled_chunk(rl, sub) << 4)) = codes;
+        if (sub == 0) e_row[rl] = (uint8_t)(e + 127);
+      }
+      if (next < nblk) load_pass(in, p, gate, up, rows, cols, nr0, nc0, rsub, sub);  // refill as consumed
     }
-    if (qt != nullptr) {
-      *reinterpret_cast<uint4*>(tile + rl * 128 + (swizzled_chunk(rl, sub) << 4)) = codes;
-      if (sub == 0) e_row[rl] = (uint8_t)(e + 127);
-    }
-  }
-  if (qt == nullptr) return;  // uniform across the CTA
 
-  // ---- direct transpose of the block (rows % 128 == 0 is guaranteed by the host)
-  __syncthreads();
-  if (tid < 32) {
-    const uint32_t w = reinterpret_cast<const uint32_t*>(e_row)[tid];
-    int m = (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24));
-    m = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)m);
-    if (tid == 0) e_max_sh = m;
-  }
-  __syncthreads();
-  const int emax = e_max_sh;
-  const int lane = tid & 31, c = tid >> 5;  // token quad = lane, 16-byte column chunk = warp
-  const uint32_t ew = reinterpret_cast<const uint32_t*>(e_row)[lane];
-  uint32_t w[4][4];
+    if (qt != nullptr) {  // uniform across the CTA
+      // ---- direct transpose of the block (rows % 128 == 0 is guaranteed by the host)
+      __syncthreads();
+      if (tid < 32) {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(e_row)[tid];
+        int m = (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24));
+        m = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)m);
+        if (tid == 0) e_max_sh = m;
+      }
+      __syncthreads();
+      const int emax = e_max_sh;
+      const int lane = tid & 31, c = tid >> 5;  // token quad = lane, 16-byte column chunk = warp
+      const uint32_t ew = reinterpret_cast<const uint32_t*>(e_row)[lane];
+      uint32_t w[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int rl = 4 * lane + i;
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + rl * 128 + (swizzled_chunk(rl, c) << 4));
-    w[i][0] = v.x;
-    w[i][1] = v.y;
-    w[i][2] = v.z;
-    w[i][3] = v.w;
-    shift_row16(w[i], emax - (int)((ew >> (8 * i)) & 0xFFu));
-  }
+      for (int i = 0; i < 4; ++i) {
+        const int rl = 4 * lane + i;
+        const uint4 v = *reinterpret_cast<const uint4*>(tile + rl * 128 + (swizzled_chunk(rl, c) << 4));
+        w[i][0] = v.x;
+        w[i][1] = v.y;
+        w[i][2] = v.z;
+        w[i][3] = v.w;
+        shift_row16(w[i], emax - (int)((ew >> (8 * i)) & 0xFFu));
+      }
 #pragma unroll
-  for (int qq = 0; qq < 4; ++qq) {
-    uint32_t o0, o1, o2, o3;
-    transpose4x4(w[0][qq], w[1][qq], w[2][qq], w[3][qq], o0, o1, o2, o3);
-    const int64_t ch = c0 + 16 * c + 4 * qq;
-    uint8_t* dst = qt + ch * rows + r0 + 4 * lane;
-    *reinterpret_cast<uint32_t*>(dst) = o0;
-    *reinterpret_cast<uint32_t*>(dst + rows) = o1;
-    *reinterpret_cast<uint32_t*>(dst + 2 * rows) = o2;
-    *reinterpret_cast<uint32_t*>(dst + 3 * rows) = o3;
+      for (int qq = 0; qq < 4; ++qq) {
+        uint32_t o0, o1, o2, o3;
+        transpose4x4(w[0][qq], w[1][qq], w[2][qq], w[3][qq], o0, o1, o2, o3);
+        const int64_t ch = c0 + 16 * c + 4 * qq;
+        uint8_t* dst = qt + ch * rows + r0 + 4 * lane;
+        *reinterpret_cast<uint32_t*>(dst) = o0;
+        *reinterpret_cast<uint32_t*>(dst + rows) = o1;
+        *reinterpret_cast<uint32_t*>(dst + 2 * rows) = o2;
+        *reinterpret_cast<uint32_t*>(dst + 3 * rows) = o3;
+      }
+      if (tid < 128) sft[(int64_t)(c0 + tid) * (rows >> 7) + (r0 >> 7)] = (uint8_t)emax;
+      __syncthreads();  // tile, e_row and e_max_sh are reused by the next block
+    }
+    if (next >= nblk) break;
+    blk = next;
   }
-  if (tid < 128) sft[(int64_t)(c0 + tid) * (rows >> 7) + (r0 >> 7)] = (uint8_t)emax;
 }
 
 // Test hooks: the device exp and SwiGLU spec on raw inputs, for cross-checks against the
@@ -180,17 +286,42 @@ __global__ void swiglu_spec_kernel(const float* __restrict__ g, const float* __r
     y[i] = swiglu_spec(g[i], u[i]);
 }
 
+// Test hook: silu of BF16 inputs through the kernel's own table path (word-pair lookup,
+// warp vote, closed forms), for an exhaustive check against the CPU spec.  Each warp
+// takes 32 consecutive words per step; lanes past the end look up 1.0 (inside the table).
+__global__ void __launch_bounds__(kThreads) silu_table_kernel(const uint32_t* __restrict__ g2, int64_t nwords,
+                                                              float2* __restrict__ out) {
+  __shared__ float silu_tab[kTab];
+  build_silu_table(silu_tab);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t step = (int64_t)gridDim.x * kThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x - lane; base < nwords; base += step) {
+    const int64_t i = base + lane;
+    const uint32_t w = i < nwords ? g2[i] : 0x3F803F80u;
+    float lo, hi;
+    uint32_t acc = 0;
+    silu_lookup2(silu_tab, w, lo, hi, acc);
+    if (__any_sync(0xFFFFFFFFu, acc != 0u)) {
+      lo = silu_fix(lo, w & 0xFFFFu, __uint_as_float(w << 16));
+      hi = silu_fix(hi, w >> 16, __uint_as_float(w & 0xFFFF0000u));
+    }
+    if (i < nwords) out[i] = make_float2(lo, hi);
+  }
+}
+
 }  // namespace
 
 fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const void* up, int64_t rows, int64_t cols,
                                 uint8_t* q, uint8_t* sf, uint8_t* qt, uint8_t* sft, cudaStream_t stream) {
-  (void)dev;
   if (rows == 0 || cols == 0) return FP8Q_OK;
-  const int64_t gx = (rows + 127) / 128;
-  if (gx > 0x7FFFFFFF || cols / 128 > 65535) return FP8Q_ERR_SHAPE;
-  dim3 grid((unsigned)gx, (unsigned)(cols / 128));
-  swiglu_quant_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(gate),
-                                                     static_cast<const uint16_t*>(up), rows, (int)cols, q, sf, qt, sft);
+  const int64_t nblk = (rows + 127) / 128 * (cols / 128);
+  if (nblk > 0x7FFFFFFF - 0x10000) return FP8Q_ERR_SHAPE;  // block indices are int32
+  const int64_t slots = (int64_t)dev.num_sms * kMinBlocks;
+  const int64_t grid = nblk < slots ? nblk : slots;
+  swiglu_quant_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(gate),
+                                                               static_cast<const uint16_t*>(up), rows, (int)cols,
+                                                               (int)nblk, q, sf, qt, sft);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -203,6 +334,12 @@ fp8q_status launch_debug_exp_spec_range(uint32_t first, int64_t n, float* out, c
 fp8q_status launch_debug_swiglu_spec(const float* g, const float* u, int64_t n, float* y, cudaStream_t stream) {
   if (n <= 0) return FP8Q_OK;
   swiglu_spec_kernel<<<1184, 256, 0, stream>>>(g, u, n, y);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+fp8q_status launch_debug_silu_bf16(const void* g, int64_t n, float* y, cudaStream_t stream) {
+  if (n <= 0) return FP8Q_OK;
+  silu_table_kernel<<<296, kThreads, 0, stream>>>(static_cast<const uint32_t*>(g), n / 2, reinterpret_cast<float2*>(y));
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

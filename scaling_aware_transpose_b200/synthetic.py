@@ -106,6 +106,22 @@ def swiglu(seed: int = 0, rows: int = 32768, cols: int = 2048) -> dict:
     return {"gate": _bf16_bits(g), "up": _bf16_bits(u)}
 
 
+
+def swiglu_wide(seed: int = 0, rows: int = 4096, cols: int = 2048) -> dict:
+    """Gate values over every BF16 binade that keeps y finite: each 1x128 gate tile draws a
+    binade B uniform in [-134, 118], each element B + {0, 1, 2} (clipped below at -133;
+    binades below -126 are BF16 subnormals), a uniform 7-bit mantissa and a random sign;
+    up ~ N(0, 1), so |y| < 2^121 * 8.  This covers tiny, table-range and huge gates in the
+    same tensor, one scale per tile."""
+    rng = np.random.default_rng(seed)
+    e = rng.integers(-134, 119, size=(rows, cols // 128, 1)) + rng.integers(0, 3, size=(rows, cols // 128, 128))
+    e = np.maximum(e, -133)
+    mant = rng.integers(0, 128, size=e.shape)
+    bits = np.where(e >= -126, ((e + 127) << 7) | mant, mant >> np.clip(-126 - e, 0, 7)).astype(np.uint16)
+    bits |= (rng.integers(0, 2, size=e.shape) << 15).astype(np.uint16)
+    u = rng.standard_normal((rows, cols), dtype=np.float32)
+    return {"gate": bits.reshape(rows, cols), "up": _bf16_bits(u)}
+
 def stress(seed: int = 0, rows: int = 65536, cols: int = 7168, lo: float = -20.0, hi: float = 12.0,
            zero_frac: float = 0.01) -> dict:
     """Range stress: each 1x128 tile is z / max|z| * 2^u with u ~ U(lo, hi) per tile

@@ -165,6 +165,12 @@ def test_debug_hook_host_errors(L):
     assert L.fp8q_debug_swiglu_spec(A, None, 16, A, None) == sat.FP8Q_ERR_NULL
     assert L.fp8q_debug_swiglu_spec(A, A, 16, A + 1, None) == sat.FP8Q_ERR_ALIGN
     assert L.fp8q_debug_swiglu_spec(None, None, 0, None, None) == sat.FP8Q_OK
+    assert L.fp8q_debug_silu_bf16(A, 15, A, None) == sat.FP8Q_ERR_ARG      # n odd
+    assert L.fp8q_debug_silu_bf16(A, -2, A, None) == sat.FP8Q_ERR_ARG
+    assert L.fp8q_debug_silu_bf16(None, 16, A, None) == sat.FP8Q_ERR_NULL
+    assert L.fp8q_debug_silu_bf16(A + 2, 16, A, None) == sat.FP8Q_ERR_ALIGN  # gate words
+    assert L.fp8q_debug_silu_bf16(A, 16, A + 4, None) == sat.FP8Q_ERR_ALIGN  # float pairs
+    assert L.fp8q_debug_silu_bf16(None, 0, None, None) == sat.FP8Q_OK
 
 
 def test_permute_host_errors(L):

@@ -2,7 +2,8 @@
 CPU oracle, over every fp32 bit pattern (non-finite inputs excluded): the fp32 -> E4M3
 conversion (round to nearest even, saturating at 448) and the SwiGLU spec's exp; plus
 the SwiGLU spec itself (y = silu(g) * u, before quantization) on a large random sample
-of finite fp32 pairs and on special values.  Inputs are generated from bit indices on
+of finite fp32 pairs and on special values; and silu of every finite BF16 value through
+the fused kernel's own table path.  Inputs are generated from bit indices on
 each side, so nothing computed by one side feeds the other."""
 import numpy as np
 import pytest
@@ -64,4 +65,27 @@ def test_swiglu_spec_matches_oracle_on_random_and_special_pairs():
     want = oracle.swiglu(g, u).view(np.uint32)
     bad = np.flatnonzero(got != want)
     assert bad.size == 0, (f"{bad.size} of {n} differ; first g={g[bad[0]]!r} u={u[bad[0]]!r}: "
+                           f"got {hex(got[bad[0]])} want {hex(want[bad[0]])}")
+
+
+@pytest.mark.parametrize("order", ["sorted", "shuffled", "ragged"])
+def test_silu_table_path_matches_oracle_on_every_finite_bf16(order):
+    """The fused SwiGLU kernel tabulates silu for BF16 inputs and uses closed forms outside
+    the table's range; every finite BF16 gate value must give the spec's fp32 silu(g).
+    Sorted, the range edges fall inside warps; shuffled, most warps that see an input
+    outside the range see only one; ragged leaves the last warp partly empty."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    bits = bits[(bits & 0x7F80) != 0x7F80].astype(np.uint16)  # finite only
+    if order == "shuffled":
+        bits = np.random.default_rng(7).permutation(bits)
+    if order == "ragged":
+        bits = bits[: 2 * 1000 + 2 * 17]
+    g = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    y = torch.empty(bits.size, dtype=torch.float32, device="cuda")
+    sat.fp8q_debug_silu_bf16(g, bits.size, y)
+    got = y.cpu().numpy().view(np.uint32)
+    gf = (bits.astype(np.uint32) << 16).view(np.float32)
+    want = oracle.swiglu(gf, np.ones_like(gf)).view(np.uint32)   # silu(g) * 1
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, (f"{bad.size} of {bits.size} differ; first g bits {hex(int(bits[bad[0]]))}: "
                            f"got {hex(got[bad[0]])} want {hex(want[bad[0]])}")

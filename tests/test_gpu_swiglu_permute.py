@@ -46,6 +46,17 @@ def test_swiglu_config_full():
     check_swiglu(synthetic.swiglu())
 
 
+def test_swiglu_persistent_ragged_rows():
+    """More blocks than resident CTAs (each CTA loops over several), last row block ragged."""
+    check_swiglu(synthetic.swiglu(rows=4100, cols=1536, seed=9), transposed=False)
+
+
+def test_swiglu_every_binade():
+    """Gates from BF16 subnormals to 2^127 in one tensor: tiny, tabulated and huge inputs
+    mixed within warps, through the persistent loop."""
+    check_swiglu(synthetic.swiglu_wide(seed=3, rows=4096, cols=2048))
+
+
 # ------------------------------------------------------------------ permute
 
 def check_permute(d, E, align):

@@ -62,3 +62,13 @@ def test_moe_combine_inputs():
     assert np.allclose(w.astype(np.float64).sum(axis=1), 1.0, atol=1e-6)
     again = synthetic.moe_combine(tokens=300, hidden=256, rows=2500, topk=8, seed=2)
     assert np.array_equal(again["y"], d["y"]) and np.array_equal(again["weights"], w)
+
+
+def test_swiglu_wide_spans_binades_and_is_seeded():
+    a = synthetic.swiglu_wide(seed=1, rows=64, cols=256)
+    b = synthetic.swiglu_wide(seed=1, rows=64, cols=256)
+    assert np.array_equal(a["gate"], b["gate"]) and np.array_equal(a["up"], b["up"])
+    g = synthetic.bf16_bits_to_f32(a["gate"])
+    assert np.isfinite(g).all() and np.abs(g).max() < 2.0 ** 121
+    mag = a["gate"] & 0x7FFF
+    assert (mag < 0x80).any() and (mag > 0x4300).any()   # subnormal and huge gates present
