@@ -16,7 +16,10 @@
 // BF16 row out.  Each thread owns 16 consecutive channels of one token (threads in
 // token-major order, so a warp reads 512 or 256 contiguous bytes of each source row and
 // writes 512 contiguous bytes), issues the loads of four slots before using any, and
-// keeps 16 fp32 accumulators.
+// keeps 16 fp32 accumulators.  For FP8 rows with top-k <= 8 (one specialisation per k)
+// the token's row indices and weights are all loaded first: a thread's 16-byte FP8 chunk
+// takes as long to arrive as the index it depends on, so this saves a round trip per four
+// slots.  BF16 rows keep the index loads inside each batch, which measured faster there.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -27,7 +30,7 @@ namespace fp8q {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kBatch = 4;  // slots whose loads are in flight together
+constexpr int kBatch = 4;  // slots whose row loads are in flight together
 
 // 2^(byte - 127) as fp32 for a UE8M0 byte in [0, 254] (byte 0 is the subnormal 2^-127).
 __device__ __forceinline__ float ue8m0_scale(uint32_t byte) {
@@ -43,7 +46,7 @@ __device__ __forceinline__ void dequant4(uint32_t w, float s, float* v) {
   v[3] = __half2float(__ushort_as_half((unsigned short)(hi >> 16))) * s;
 }
 
-template <bool kFp8>
+template <bool kFp8, int kK>
 __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t* __restrict__ y,
                                                                    const uint8_t* __restrict__ y_sf, int64_t rows,
                                                                    int hidden, const int32_t* __restrict__ row_id_map,
@@ -60,54 +63,102 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = -0.0f;
 
-  for (int s0 = 0; s0 < topk; s0 += kBatch) {
-    uint4 d0[kBatch], d1[kBatch];  // 16 codes, or 16 bf16 in two halves
-    float ws[kBatch], sc[kBatch];
-    bool use[kBatch];
+  if constexpr (kFp8 && kK > 0) {
+    // FP8 rows, top-k fixed at compile time: the token's indices and weights first, in one
+    // round trip, then the rows, kBatch slots at a time.
+    {
+      int64_t rr[kK];
+      float wg[kK];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int s = s0 + b;
-      use[b] = false;
-      ws[b] = 1.0f;
-      sc[b] = 1.0f;
-      d0[b] = d1[b] = make_uint4(0u, 0u, 0u, 0u);
-      if (s < topk) {
-        const int64_t r = __ldg(row_id_map + t * topk + s);
-        if (r < 0 || r >= rows) {
-          record_status(status, FP8Q_ERR_DEVICE);  // the slot is skipped
-        } else {
-          use[b] = true;
-          if (weights != nullptr) ws[b] = __ldg(weights + t * topk + s);
-          if (kFp8) {
-            d0[b] = __ldg(reinterpret_cast<const uint4*>(y + r * hidden + h0));
-            sc[b] = ue8m0_scale(__ldg(y_sf + r * ntile + (h0 >> 7)));
-          } else {
-            const uint4* src = reinterpret_cast<const uint4*>(y + (r * hidden + h0) * 2);
-            d0[b] = __ldg(src);
-            d1[b] = __ldg(src + 1);
+      for (int s = 0; s < kK; ++s) {
+        rr[s] = __ldg(row_id_map + t * kK + s);
+        wg[s] = weights != nullptr ? __ldg(weights + t * kK + s) : 1.0f;
+      }
+#pragma unroll
+      for (int s0 = 0; s0 < kK; s0 += kBatch) {
+        uint4 d[kBatch];
+        float sc[kBatch];
+        bool use[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          const int s = s0 + b;
+          const int64_t r = s < kK ? rr[s] : 0;
+          use[b] = false;
+          sc[b] = 1.0f;
+          d[b] = make_uint4(0u, 0u, 0u, 0u);
+          if (s < kK) {
+            if (r < 0 || r >= rows) {
+              record_status(status, FP8Q_ERR_DEVICE);  // the slot is skipped
+            } else {
+              use[b] = true;
+              d[b] = __ldg(reinterpret_cast<const uint4*>(y + r * hidden + h0));
+              sc[b] = ue8m0_scale(__ldg(y_sf + r * ntile + (h0 >> 7)));
+            }
           }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          if (!use[b]) continue;
+          float v[16];
+          dequant4(d[b].x, sc[b], v);
+          dequant4(d[b].y, sc[b], v + 4);
+          dequant4(d[b].z, sc[b], v + 8);
+          dequant4(d[b].w, sc[b], v + 12);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = __fmaf_rn(wg[s0 + b < kK ? s0 + b : 0], v[i], acc[i]);
         }
       }
     }
+  } else {  // BF16 rows, or FP8 rows with top-k > 8
+    for (int s0 = 0; s0 < topk; s0 += kBatch) {
+      uint4 d0[kBatch], d1[kBatch];  // 16 codes, or 16 bf16 in two halves
+      float ws[kBatch], sc[kBatch];
+      bool use[kBatch];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      if (!use[b]) continue;
-      float v[16];
-      if (kFp8) {
-        dequant4(d0[b].x, sc[b], v);
-        dequant4(d0[b].y, sc[b], v + 4);
-        dequant4(d0[b].z, sc[b], v + 8);
-        dequant4(d0[b].w, sc[b], v + 12);
-      } else {
-        const uint32_t wd[8] = {d0[b].x, d0[b].y, d0[b].z, d0[b].w, d1[b].x, d1[b].y, d1[b].z, d1[b].w};
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          v[2 * k] = __uint_as_float(wd[k] << 16);
-          v[2 * k + 1] = __uint_as_float(wd[k] & 0xFFFF0000u);
+      for (int b = 0; b < kBatch; ++b) {
+        const int s = s0 + b;
+        use[b] = false;
+        ws[b] = 1.0f;
+        sc[b] = 1.0f;
+        d0[b] = d1[b] = make_uint4(0u, 0u, 0u, 0u);
+        if (s < topk) {
+          const int64_t r = __ldg(row_id_map + t * topk + s);
+          if (r < 0 || r >= rows) {
+            record_status(status, FP8Q_ERR_DEVICE);  // the slot is skipped
+          } else {
+            use[b] = true;
+            if (weights != nullptr) ws[b] = __ldg(weights + t * topk + s);
+            if (kFp8) {
+              d0[b] = __ldg(reinterpret_cast<const uint4*>(y + r * hidden + h0));
+              sc[b] = ue8m0_scale(__ldg(y_sf + r * ntile + (h0 >> 7)));
+            } else {
+              const uint4* src = reinterpret_cast<const uint4*>(y + (r * hidden + h0) * 2);
+              d0[b] = __ldg(src);
+              d1[b] = __ldg(src + 1);
+            }
+          }
         }
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = __fmaf_rn(ws[b], v[i], acc[i]);
+      for (int b = 0; b < kBatch; ++b) {
+        if (!use[b]) continue;
+        float v[16];
+        if (kFp8) {
+          dequant4(d0[b].x, sc[b], v);
+          dequant4(d0[b].y, sc[b], v + 4);
+          dequant4(d0[b].z, sc[b], v + 8);
+          dequant4(d0[b].w, sc[b], v + 12);
+        } else {
+          const uint32_t wd[8] = {d0[b].x, d0[b].y, d0[b].z, d0[b].w, d1[b].x, d1[b].y, d1[b].z, d1[b].w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            v[2 * k] = __uint_as_float(wd[k] << 16);
+            v[2 * k + 1] = __uint_as_float(wd[k] & 0xFFFF0000u);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = __fmaf_rn(ws[b], v[i], acc[i]);
+      }
     }
   }
   uint32_t o[8];
@@ -121,6 +172,25 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
   dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+struct UnpermuteArgs {
+  const uint8_t* y;
+  const uint8_t* y_sf;
+  int64_t rows;
+  int hidden;
+  const int32_t* row_id_map;
+  const float* weights;
+  int64_t tokens;
+  int topk;
+  uint16_t* out;
+  int* status;
+};
+
+template <bool kFp8, int kK>
+void launch_k(const UnpermuteArgs& a, unsigned blocks, cudaStream_t stream) {
+  unpermute_unpad_kernel<kFp8, kK><<<blocks, kThreads, 0, stream>>>(a.y, a.y_sf, a.rows, a.hidden, a.row_id_map,
+                                                                    a.weights, a.tokens, a.topk, a.out, a.status);
+}
+
 }  // namespace
 
 fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const uint8_t* y_sf, int64_t rows,
@@ -128,16 +198,26 @@ fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const u
                                    int32_t topk, void* out, cudaStream_t stream) {
   const int64_t threads = tokens * (hidden / 16);
   if (threads == 0) return FP8Q_OK;
-  const int64_t blocks = (threads + kThreads - 1) / kThreads;
-  if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  if (y_sf)
-    unpermute_unpad_kernel<true><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(y), y_sf, rows, (int)hidden, row_id_map, weights, tokens, topk,
-        static_cast<uint16_t*>(out), dev.status);
-  else
-    unpermute_unpad_kernel<false><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(y), nullptr, rows, (int)hidden, row_id_map, weights, tokens, topk,
-        static_cast<uint16_t*>(out), dev.status);
+  const int64_t blocks64 = (threads + kThreads - 1) / kThreads;
+  if (blocks64 > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const unsigned blocks = (unsigned)blocks64;
+  const UnpermuteArgs a{static_cast<const uint8_t*>(y), y_sf, rows, (int)hidden, row_id_map, weights, tokens, topk,
+                        static_cast<uint16_t*>(out), dev.status};
+  if (y_sf == nullptr) {
+    launch_k<false, 0>(a, blocks, stream);
+  } else {
+    switch (topk) {
+      case 1: launch_k<true, 1>(a, blocks, stream); break;
+      case 2: launch_k<true, 2>(a, blocks, stream); break;
+      case 3: launch_k<true, 3>(a, blocks, stream); break;
+      case 4: launch_k<true, 4>(a, blocks, stream); break;
+      case 5: launch_k<true, 5>(a, blocks, stream); break;
+      case 6: launch_k<true, 6>(a, blocks, stream); break;
+      case 7: launch_k<true, 7>(a, blocks, stream); break;
+      case 8: launch_k<true, 8>(a, blocks, stream); break;
+      default: launch_k<true, 0>(a, blocks, stream); break;
+    }
+  }
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

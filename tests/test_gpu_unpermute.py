@@ -1,6 +1,6 @@
 """GPU parity of the fused unpermute + unpad (combine side of the permute) against the
 CPU oracle, byte for byte: BF16 and FP8 expert rows, routing weights and unit weights,
-K = 1..8, ragged hidden sizes, the permute round trip, the full MoE workload, and bad
+K = 1..8 (each its own FP8 specialisation) and 12, 16, ragged hidden sizes, the permute round trip, the full MoE workload, and bad
 row indices reported through the status word."""
 import numpy as np
 import pytest
@@ -27,7 +27,8 @@ def case(T, H, K, R, seed, fp8):
 
 @pytest.mark.parametrize("fp8", [False, True])
 @pytest.mark.parametrize("weighted", [False, True])
-@pytest.mark.parametrize("T,H,K", [(1, 128, 1), (37, 384, 2), (64, 640, 3), (100, 1152, 8), (257, 256, 5), (33, 7168, 8)])
+@pytest.mark.parametrize("T,H,K", [(1, 128, 1), (37, 384, 2), (64, 640, 3), (40, 512, 4), (257, 256, 5), (29, 896, 6),
+                                   (50, 256, 7), (100, 1152, 8), (33, 7168, 8), (45, 384, 12), (20, 1024, 16)])
 def test_matches_oracle(fp8, weighted, T, H, K):
     R = T * K + 50
     y, sf, rmap, w = case(T, H, K, R, seed=T + H + K, fp8=fp8)
@@ -74,6 +75,17 @@ def test_bad_row_index_sets_device_status():
     rmap = torch.tensor([0, -5], dtype=torch.int32, device="cuda")
     sat.unpermute_unpad(y, rmap, 2)
     assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE
+    assert sat.fp8q_last_device_status() == 0
+
+
+def test_bad_row_index_sets_device_status_fp8():
+    """The FP8 kernels (one per top-k up to 8, a generic one above) report a bad index too."""
+    q = torch.zeros((64, 256), dtype=torch.uint8, device="cuda")
+    sf = torch.full((64, 2), 127, dtype=torch.uint8, device="cuda")
+    for K, bad in ((2, [0, 1, 64, 3]), (8, list(range(15)) + [-1]), (12, list(range(23)) + [99])):
+        rmap = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        sat.unpermute_unpad(q, rmap, K, None, sf)
+        assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE, K
     assert sat.fp8q_last_device_status() == 0
 
 
