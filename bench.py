@@ -60,7 +60,7 @@ def kernel_sources(kind: str):
     csrc = os.path.join(ROOT, "scaling_aware_transpose_b200", "csrc")
     main = {"quantize": "quantize_rowwise.cu", "direct": "direct_transpose.cu", "swiglu": "swiglu_quant.cu",
             "permute": "permute_pad_quant.cu", "rowwise_colwise": "quantize_rowwise_colwise.cu",
-            "unpermute": "unpermute_unpad.cu", "mx32": "mx32.cu"}[kind]
+            "unpermute": "unpermute_unpad.cu", "unpermute_fp8": "unpermute_unpad.cu", "mx32": "mx32.cu"}[kind]
     return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")]
 
 
@@ -665,7 +665,7 @@ def run_profile(args):
         qt = torch.empty((C, R), dtype=torch.uint8, device="cuda")
         sft = torch.empty((C, R // 128), dtype=torch.uint8, device="cuda")
         calls = {"swiglu": lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, qt, sft)}
-    elif args.profile == "unpermute":
+    elif args.profile in ("unpermute", "unpermute_fp8"):
         d = synthetic.moe()
         x = synthetic.to_torch_bf16(d["x"]).cuda()
         idx = torch.from_numpy(d["topk_idx"]).cuda()
@@ -675,7 +675,8 @@ def run_profile(args):
         c = synthetic.moe_combine(rows=R, topk=K)
         y = synthetic.to_torch_bf16(c["y"]).cuda()
         wts = torch.from_numpy(c["weights"]).cuda()
-        calls = {"unpermute": lambda: sat.unpermute_unpad(y, rmap, K, wts)}
+        calls = {"unpermute": lambda: sat.unpermute_unpad(y, rmap, K, wts),
+                 "unpermute_fp8": lambda: sat.unpermute_unpad(pq, rmap, K, None, psf)}
     else:  # permute
         d = synthetic.moe()
         x = synthetic.to_torch_bf16(d["x"]).cuda()
@@ -701,7 +702,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
     ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise",
-                                          "unpermute", "mx32", "permute_fp8"],
+                                          "unpermute", "unpermute_fp8", "mx32", "permute_fp8"],
                     default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)
