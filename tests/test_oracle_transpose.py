@@ -161,3 +161,35 @@ def test_error_report_runs(tiny_q):
         assert 0.0 <= oracle.rel_rms(arr, x) < 0.2
         assert 0.0 <= oracle.calc_diff(arr, x) < 0.05
     assert oracle.rel_rms(v, v) == 0.0
+
+
+def _row_rel_rms(a, ref):
+    num = np.sqrt(((a - ref) ** 2).sum(axis=1))
+    den = np.sqrt((ref ** 2).sum(axis=1))
+    return num[den > 0] / den[den > 0]
+
+
+@pytest.mark.parametrize("recipe", ["dense", "stress"])
+def test_error_report_direct_vs_double_quantization(recipe):
+    """The error report on 1024 rows of the dense and range-stress recipes (reported
+    numbers; run with -s to print them).  The column-wise result of the direct transpose
+    stays within the row-wise quantization's own error of X, while a requantization with
+    fresh non-power-of-two column scales (the double quantization the method avoids)
+    adds two orders of magnitude more error relative to the row-wise values."""
+    d = synthetic.dense(seed=0, rows=1024) if recipe == "dense" else synthetic.stress(seed=0, rows=1024)
+    x = synthetic.bf16_bits_to_f32(d["x"]).astype(np.float64)
+    q, sf = oracle.quantize_rowwise(d["x"])
+    v = oracle.dequant_rowwise(q, sf)
+    res = {"row-wise": v,
+           "direct": oracle.dequant_colwise(*oracle.direct_transpose(q, sf)),
+           "naive (pow2)": oracle.dequant_colwise(*oracle.naive_transpose(q, sf)),
+           "naive (fp32 amax/448)": oracle.naive_fp32_colwise(v)}
+    print(f"\n{recipe} [1024x7168]: rel RMS vs X | vs row-wise values | calc_diff vs X | per-row rel RMS vs X p50 / p99")
+    for name, a in res.items():
+        rr = _row_rel_rms(a, x)
+        print(f"  {name:22s} {oracle.rel_rms(a, x):.4e} | {oracle.rel_rms(a, v):.4e} | {oracle.calc_diff(a, x):.3e} | "
+              f"{np.percentile(rr, 50):.3e} / {np.percentile(rr, 99):.3e}")
+    extra_direct = oracle.rel_rms(res["direct"], v)
+    extra_fp32 = oracle.rel_rms(res["naive (fp32 amax/448)"], v)
+    assert extra_direct * 100 < extra_fp32
+    assert oracle.rel_rms(res["direct"], x) < oracle.rel_rms(res["naive (fp32 amax/448)"], x)
