@@ -2,11 +2,11 @@
 //
 // FP8-Flow-MoE review, 核心方法 (Fused SwiGLU+Quantization): the activation output is
 // produced directly in FP8 at the activation boundary instead of a BF16 tensor followed
-// by a separate quantize.  Here each CTA owns one 128x128 block: it reads gate and up
-// (bf16) once, computes y = silu(gate) * up in fp32, quantizes each 1x128 row tile with
-// a power-of-two scale, writes the row-wise codes and scales, and, when asked, converts
-// the block to the column-wise layout with the scaling-aware shift before any byte
-// leaves the SM.
+// by a separate quantize.  Here a CTA works on one 128x128 block at a time: it reads
+// gate and up (bf16) once, computes y = silu(gate) * up in fp32, quantizes each 1x128
+// row tile with a power-of-two scale, writes the row-wise codes and scales, and, when
+// asked, converts the block to the column-wise layout with the scaling-aware shift
+// before any byte leaves the SM.
 //
 // Arithmetic spec of y (every step one IEEE fp32 operation, round to nearest even, no
 // contraction; identical on every implementation of this spec):
