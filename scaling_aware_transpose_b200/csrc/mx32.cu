@@ -15,11 +15,12 @@
 //
 // direct_transpose_mx32_kernel: the 128x128 block-per-CTA direct transpose with 16 MX
 // blocks per CTA tile.  Each row's four scale bytes (one per 32-column group) move as one
-// 32-bit word; every warp computes the Smax of all sixteen (row group, column group)
-// blocks itself with single-instruction warp max reductions (__reduce_max_sync), so one
-// barrier suffices as in the 128 kernel.  The shift of a 16-byte row chunk uses its
-// own 32x32 block's k; staging and the byte transpose (8 tokens x 8 channels per lane)
-// are those of the 128 kernel.
+// 32-bit word.  The four warps that load the scale words each reduce their own row group
+// (one single-instruction warp max per column group, __reduce_max_sync) and publish one
+// packed word before the kernel's one barrier; every thread then assembles the two words
+// of maxima it needs with byte permutes.  The shift of a 16-byte row chunk uses its own
+// 32x32 block's k; staging and the byte transpose (8 tokens x 8 channels per lane) are
+// those of the 128 kernel.
 #include "common.cuh"
 #include "launch.h"
 
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
                                                                           uint8_t* __restrict__ sft) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ uint32_t e_row[128];  // 4 scale bytes of the row: column groups 0..3 of this tile
+  __shared__ __align__(16) uint32_t smax_rg[4];  // row group rg: Smax byte of column groups 0..3
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const int ngr = cols >> 5;  // scale bytes per row
@@ -91,25 +93,26 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   uint4 v[kPasses];
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) v[p] = __ldg(reinterpret_cast<const uint4*>(qb + (p * 32 + rsub) * cols) + sub);
-  // the row's 4 scale bytes: 4-byte aligned (rows of cols/32 bytes, cols % 128 == 0)
-  if (tid < 128) e_row[tid] = __ldg(reinterpret_cast<const uint32_t*>(sf + (r0 + tid) * ngr + (c0 >> 5)));
+  // The row's 4 scale bytes (4-byte aligned: rows of cols/32 bytes, cols % 128 == 0).
+  // Warp rg < 4 loads the 32 rows of row group rg and reduces their Smax per column group
+  // with single-instruction warp reductions, one packed word per row group.
+  if (tid < 128) {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(sf + (r0 + tid) * ngr + (c0 >> 5)));
+    e_row[tid] = w;
+    uint32_t m = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) m |= __reduce_max_sync(0xFFFFFFFFu, (w >> (8 * c)) & 0xFFu) << (8 * c);
+    if ((tid & 31) == 0) smax_rg[tid >> 5] = m;
+  }
   __syncthreads();
-  // Smax of every (row group, column group) with single-instruction warp reductions; keep
-  // the two packed words this thread needs: its own column group over the row groups,
-  // and the SF^T channel's column group over the row groups.
+  // The two words this thread needs, byte rg = Smax of (row group rg, column group): its
+  // own chunks' column group, and the column group of SF^T channel c0 + tid.
   const int cg = sub >> 1;            // 32-column group of this thread's 16-byte chunks
   const int cg_t = (tid >> 5) & 3;    // column group of channel c0 + tid (SF^T word)
-  uint32_t smax_mine = 0, smax_sft = 0;
-#pragma unroll
-  for (int rg = 0; rg < 4; ++rg) {
-    const uint32_t w = e_row[32 * rg + (tid & 31)];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, (w >> (8 * c)) & 0xFFu);
-      smax_mine |= (c == cg ? m : 0u) << (8 * rg);
-      smax_sft |= (c == cg_t ? m : 0u) << (8 * rg);
-    }
-  }
+  const uint4 sm = *reinterpret_cast<const uint4*>(smax_rg);
+  const uint32_t sel = (uint32_t)cg | (uint32_t)(cg + 4) << 4, sel_t = (uint32_t)cg_t | (uint32_t)(cg_t + 4) << 4;
+  const uint32_t smax_mine = __byte_perm(__byte_perm(sm.x, sm.y, sel), __byte_perm(sm.z, sm.w, sel), 0x5410);
+  const uint32_t smax_sft = __byte_perm(__byte_perm(sm.x, sm.y, sel_t), __byte_perm(sm.z, sm.w, sel_t), 0x5410);
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
     const int rl = p * 32 + rsub;  // row group p
