@@ -10,8 +10,10 @@
 //
 // Launches: (1) per-chunk expert histograms, (2) one CTA scans them into padded expert
 // offsets and per-chunk bases, (3) stable ranks within each chunk with __match_any_sync
-// (eight warps per chunk for up to 512 experts, one warp beyond), (4) the streaming scatter-quantize over all (token, tile) pairs, whose
-// trailing CTAs zero-fill the padding rows.  Workspace: counts[C][E], bases[C][E], totals[E].
+// (eight warps per chunk for up to 512 experts, one warp beyond), (4) the streaming
+// scatter-quantize over all (token, tile) pairs, whose trailing CTAs zero-fill the
+// padding rows.  (2)-(4) are programmatic dependent launches that overlap the tail of
+// their predecessor (see pdl_wait).  Workspace: counts[C][E], bases[C][E], totals[E].
 // The FP8-input variant (the dispatch already delivered row-wise codes and scales) shares
 // (1)-(3) and the padding; its step (4) copies each token's codes and scale bytes to its
 // rows.
@@ -22,6 +24,16 @@ namespace fp8q {
 namespace {
 
 constexpr int kChunk = 1024;  // (t, s) pairs per chunk, in row-major order
+
+// Programmatic dependent launch (sm_90 and later): the scan, rank and scatter launches
+// carry the programmatic-stream-serialization attribute, so each may be scheduled while
+// its predecessor in the chain still runs.  pdl_wait() returns once the predecessor grid
+// has completed and its writes are visible (a hardware dependency, not a spin loop);
+// pdl_trigger() lets the successor be scheduled.  In a launch without the attribute both
+// are no-ops.  The first kernel of a call (the histogram) is launched plainly, so no part
+// of a call overlaps work queued before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 constexpr int kMaxExperts = 4096;
 
 int64_t num_chunks(int64_t tokens, int32_t topk) { return (tokens * topk + kChunk - 1) / kChunk; }
@@ -29,6 +41,7 @@ int64_t num_chunks(int64_t tokens, int32_t topk) { return (tokens * topk + kChun
 __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
                                                     int32_t* __restrict__ counts, int* status) {
   extern __shared__ int32_t hist[];
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int64_t p0 = (int64_t)blockIdx.x * kChunk;
@@ -70,6 +83,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
   __shared__ int32_t s_off[kMaxExperts];
   __shared__ int32_t s_warp[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  pdl_wait();  // the histograms
   for (int e = warp; e < E; e += 32) {
     int32_t acc = 0;
     for (int64_t c0 = 0; c0 < C; c0 += 8 * 32) {
@@ -141,6 +156,8 @@ __global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ id
     const int64_t p = p0 + i * 32 + lane;
     ids[i] = p < npairs ? __ldg(idx + p) : -1;
   }
+  pdl_trigger();
+  pdl_wait();  // the bases
   for (int e = lane; e < E; e += 32) run[e] = bases[(int64_t)blockIdx.x * E + e];
   __syncwarp();
 #pragma unroll 4
@@ -184,6 +201,7 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
     const int64_t p = p0 + i * 32 + lane;
     ids[i] = p < npairs ? __ldg(idx + p) : -1;
   }
+  pdl_trigger();
   for (int e = tid; e < kRankWarps * E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
   int32_t* mine = s_cnt + w * E;
@@ -197,6 +215,7 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
     __syncwarp();
   }
   __syncthreads();
+  pdl_wait();  // the bases
   for (int e = tid; e < E; e += blockDim.x) {
     int32_t run = bases[(int64_t)blockIdx.x * E + e];
 #pragma unroll
@@ -277,6 +296,7 @@ __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* _
                                                                   const int32_t* __restrict__ offsets,
                                                                   const int32_t* __restrict__ totals) {
   if ((int64_t)blockIdx.x >= scatter_ctas) {
+    pdl_wait();  // the offsets
     pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
              reinterpret_cast<uint8_t*>(q), sf);
     return;
@@ -296,6 +316,8 @@ __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* _
       v0[u] = v1[u] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  uint2 lo[kSUnroll], hi[kSUnroll];
+  int e[kSUnroll];
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
     uint32_t m = maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(v0[u].x, v0[u].y), maxabs_bf16x2(v0[u].z, v0[u].w)),
@@ -303,20 +325,24 @@ __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* _
     m = maxabs_bf16x2(m, __byte_perm(m, 0u, 0x1032)) & 0x7FFFu;
 #pragma unroll
     for (int o = 4; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    e[u] = bf16_tile_exponent(m);
+    const float s = exp2_neg(e[u]);
+    lo[u] = make_uint2(encode4(v0[u].x, v0[u].y, s), encode4(v0[u].z, v0[u].w, s));
+    hi[u] = make_uint2(encode4(v1[u].x, v1[u].y, s), encode4(v1[u].z, v1[u].w, s));
+  }
+  pdl_wait();  // the row ids: everything above overlaps the routing
+#pragma unroll
+  for (int u = 0; u < kSUnroll; ++u) {
     if (tile[u] >= n_tiles) continue;
-    const int e = bf16_tile_exponent(m);
-    const float s = exp2_neg(e);
-    const uint2 lo = make_uint2(encode4(v0[u].x, v0[u].y, s), encode4(v0[u].z, v0[u].w, s));
-    const uint2 hi = make_uint2(encode4(v1[u].x, v1[u].y, s), encode4(v1[u].z, v1[u].w, s));
     const int64_t t = tile[u] / ncb;
     const int j = (int)(tile[u] - t * ncb);
     for (int k = 0; k < topk; ++k) {
       const int32_t row = __ldg(row_id_map + t * topk + k);
       if (row < 0) continue;
       uint2* dst = q + ((int64_t)row * ncb + j) * 16;
-      dst[sub] = lo;
-      dst[8 + sub] = hi;
-      if (sub == 0) sf[(int64_t)row * ncb + j] = (uint8_t)(e + 127);
+      dst[sub] = lo[u];
+      dst[8 + sub] = hi[u];
+      if (sub == 0) sf[(int64_t)row * ncb + j] = (uint8_t)(e[u] + 127);
     }
   }
 }
@@ -333,6 +359,7 @@ __global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __
                                                                  int pad_slots, const int32_t* __restrict__ offsets,
                                                                  const int32_t* __restrict__ totals) {
   if ((int64_t)blockIdx.x >= scatter_ctas) {
+    pdl_wait();  // the offsets
     pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
              reinterpret_cast<uint8_t*>(q), sf);
     return;
@@ -353,6 +380,7 @@ __global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __
       if (sub == 0) e[u] = __ldg(xsf + tile[u]);
     }
   }
+  pdl_wait();  // the row ids
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
     if (tile[u] >= n_tiles) continue;
@@ -376,6 +404,23 @@ size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts
 
 namespace {
 
+// A launch that may begin while the previous kernel in the stream finishes (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                         Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Steps (1)-(3): offsets, per-chunk bases, row ids.
 fp8q_status route(const DeviceInfo& dev, int64_t tokens, const int32_t* topk_idx, int32_t topk, int E, int32_t align,
                   int32_t* expert_offsets, int32_t* row_id_map, int32_t* counts, int32_t* bases, int32_t* totals,
@@ -385,14 +430,16 @@ fp8q_status route(const DeviceInfo& dev, int64_t tokens, const int32_t* topk_idx
   const size_t hist_smem = (size_t)E * sizeof(int32_t);
   count_kernel<<<(unsigned)C, 256, hist_smem, stream>>>(topk_idx, npairs, E, counts, dev.status);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  scan_kernel<<<1, 1024, 0, stream>>>(counts, C, E, align, expert_offsets, bases, totals);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  if (E <= kRankMultiMaxE)
-    rank_multi_kernel<<<(unsigned)C, kRankWarps * 32, (size_t)kRankWarps * E * sizeof(int32_t), stream>>>(
-        topk_idx, npairs, E, bases, row_id_map);
-  else
-    rank_kernel<<<(unsigned)C, 32, hist_smem, stream>>>(topk_idx, npairs, E, bases, row_id_map);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  if (launch_after(scan_kernel, 1, 1024, 0, stream, (const int32_t*)counts, C, E, (int)align, expert_offsets, bases,
+                   totals) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  const cudaError_t rc =
+      E <= kRankMultiMaxE
+          ? launch_after(rank_multi_kernel, (unsigned)C, kRankWarps * 32, (size_t)kRankWarps * E * sizeof(int32_t),
+                         stream, topk_idx, npairs, E, (const int32_t*)bases, row_id_map)
+          : launch_after(rank_kernel, (unsigned)C, 32, hist_smem, stream, topk_idx, npairs, E, (const int32_t*)bases,
+                         row_id_map);
+  return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 // xq/xsf != nullptr: FP8-input payload; else quantize x.
@@ -421,15 +468,17 @@ fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq,
   const int pad_slots = (align - 1 + kPadRowsPerCta - 1) / kPadRowsPerCta;  // 0 when align == 1
   const int64_t blocks = scatter_ctas + (int64_t)E * pad_slots;
   if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  if (xq)
-    scatter_copy_kernel<<<(unsigned)blocks, kSThreads, 0, stream>>>(
-        reinterpret_cast<const uint4*>(xq), xsf, tokens, ncb, row_id_map, topk, reinterpret_cast<uint4*>(q), sf,
-        scatter_ctas, pad_slots, expert_offsets, totals);
-  else
-    scatter_quant_kernel<<<(unsigned)blocks, kSThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), tokens, ncb, row_id_map, topk, reinterpret_cast<uint2*>(q), sf, scatter_ctas,
-        pad_slots, expert_offsets, totals);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  const int32_t* rmap = row_id_map;
+  const int32_t* offs = expert_offsets;
+  const int32_t* tots = totals;
+  const cudaError_t rc =
+      xq ? launch_after(scatter_copy_kernel, (unsigned)blocks, kSThreads, 0, stream,
+                        reinterpret_cast<const uint4*>(xq), xsf, tokens, ncb, rmap, (int)topk,
+                        reinterpret_cast<uint4*>(q), sf, scatter_ctas, pad_slots, offs, tots)
+         : launch_after(scatter_quant_kernel, (unsigned)blocks, kSThreads, 0, stream, static_cast<const uint4*>(x),
+                        tokens, ncb, rmap, (int)topk, reinterpret_cast<uint2*>(q), sf, scatter_ctas, pad_slots, offs,
+                        tots);
+  return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 }  // namespace
