@@ -70,6 +70,33 @@ def test_swiglu_close_to_double_reference():
     assert np.all(np.abs(y - ref) <= 4 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64) + 1e-45)
 
 
+def test_silu_closed_forms_over_every_bf16_gate():
+    """On BF16 gates the spec's silu(g) = g / (1 + exp(-g)) reduces to one IEEE operation
+    outside one magnitude range: below BF16 0x33C1 the denominator rounds to exactly 2
+    (silu = RN(g/2)); from 89 up exp(-g) <= 2^-24 and the denominator rounds to 1
+    (silu = g, true already from 16.75); from -89 down exp(-g) overflows to +inf
+    (silu = -0).  These are the facts a kernel may use to tabulate only the rest; the
+    thresholds are tight at the low end (0x33C1 itself breaks the first rule)."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    bits = bits[(bits & 0x7F80) != 0x7F80]
+    g = (bits << 16).view(np.float32)
+    s = oracle.swiglu(g, np.ones_like(g)).view(np.uint32)
+    mag, neg = bits & 0x7FFF, bits >> 15
+    tiny = mag < 0x33C1
+    half = (g[tiny].astype(np.float64) * 0.5).astype(np.float32)   # exact product, one rounding
+    assert np.array_equal(s[tiny], half.view(np.uint32))
+    big_pos = (mag >= 0x4186) & (neg == 0)
+    assert np.array_equal(s[big_pos], g[big_pos].view(np.uint32))
+    big_neg = (mag >= 0x42B2) & (neg == 1)
+    assert (s[big_neg] == 0x80000000).all()
+    # the low threshold is tight: the positive gate 0x33C1 does not give RN(g/2)
+    g1 = np.array([(0x33C1 << 16)], np.uint32).view(np.float32)
+    assert oracle.swiglu(g1, np.ones(1, np.float32)).view(np.uint32)[0] != (g1 * np.float32(0.5)).view(np.uint32)[0]
+    # and just below 89 the negative side is not yet -0
+    g2 = np.array([(0xC2B1 << 16)], np.uint32).view(np.float32)
+    assert oracle.swiglu(g2, np.ones(1, np.float32)).view(np.uint32)[0] != 0x80000000
+
+
 def test_swiglu_quant_is_quantize_of_swiglu_then_direct():
     d = synthetic.swiglu(rows=256, cols=384, seed=10)
     q, sf, qt, sft = oracle.swiglu_quant(d["gate"], d["up"])
