@@ -246,23 +246,6 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
   }
 }
 
-__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-// Tile exponent from the BF16 amax bit pattern (see quantize_rowwise.cu): e = E - 135,
-// plus one when the mantissa exceeds 0x60; 0 for a zero tile; clamped at -127.
-__device__ __forceinline__ int bf16_tile_exponent(uint32_t amax16) {
-  const int e = (int)(amax16 >> 7) - 135 + ((amax16 & 0x7Fu) > 0x60u ? 1 : 0);
-  return amax16 == 0u ? 0 : max(e, -127);
-}
-__device__ __forceinline__ uint32_t encode4(uint32_t a, uint32_t b, float s) {
-  const float f0 = __uint_as_float(a << 16) * s, f1 = __uint_as_float(a & 0xFFFF0000u) * s;
-  const float f2 = __uint_as_float(b << 16) * s, f3 = __uint_as_float(b & 0xFFFF0000u) * s;
-  return __byte_perm(cvt_e4m3x2_f32(f0, f1), cvt_e4m3x2_f32(f2, f3), 0x5410);
-}
-
 // Padding rows: CTA slot `slot` of expert e zeroes rows offsets[e] + totals[e] + 8*slot ..
 // (at most 8 rows, never past offsets[e+1]): codes 0x00, scale byte 127.  Run by the
 // trailing CTAs of the scatter launch (E x ceil((align-1)/8) of them).
