@@ -91,3 +91,23 @@ def test_reference_arm_other_ranks_do_nothing(capsys, monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--steps", "1"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_every_profile_choice_names_existing_sources():
+    """Each --profile choice that has a summary under profiles/ maps to kernel sources that
+    exist, so a summary's source hash can always be recomputed."""
+    for kind in ("quantize", "direct", "swiglu", "permute", "rowwise_colwise", "unpermute", "unpermute_fp8", "mx32"):
+        paths = bench.kernel_sources(kind)
+        assert paths and all(os.path.exists(p) for p in paths), kind
+    assert bench.kernel_sources("unpermute_fp8") == bench.kernel_sources("unpermute")
+
+
+def test_profile_summaries_carry_command_and_hash():
+    """Every committed ncu summary names the command that made it and a source hash."""
+    d = os.path.join(bench.ROOT, "profiles")
+    for name in sorted(os.listdir(d)):
+        txt = open(os.path.join(d, name)).read()
+        assert "--clock-control none" in txt, name
+        if name.startswith("launches_"):
+            continue
+        assert "source_sha256:" in txt and "dram_bytes_per_launch:" in txt, name
