@@ -127,7 +127,8 @@ fp8q_status fp8q_naive_transpose(const uint8_t *q, const uint8_t *sf, int64_t ro
 fp8q_status fp8q_swiglu_quant(const void *gate, const void *up, int64_t rows, int64_t cols, uint8_t *q,
                               uint8_t *sf, uint8_t *qt, uint8_t *sft, fp8q_stream_t stream);
 
-/* Bytes of device workspace fp8q_permute_pad_quant needs. */
+/* Bytes of device workspace fp8q_permute_pad_quant needs; 0 for arguments no permute
+ * accepts (negative tokens, topk < 1, num_experts < 1, tokens*topk beyond 2^31 - 1). */
 size_t fp8q_permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts);
 
 /* Fused permute + pad + row-wise quantize (FP8-Flow-MoE 核心方法: Fused
@@ -144,7 +145,8 @@ size_t fp8q_permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_ex
  *   expert_offsets : out int32 [num_experts + 1], exclusive scan of padded sizes.
  *   row_id_map     : out int32 [tokens*topk], destination row of pair (t, s).
  *   workspace      : device, >= fp8q_permute_workspace_bytes(...), 16-byte aligned.
- *   align in [1, 4096]; num_experts in [1, 4096]; topk in [1, 64].
+ *   align in [1, 4096]; num_experts in [1, 4096]; topk in [1, 64]; tokens*topk and
+ *   max_out_rows at most 2^31 - 1 (row ids are int32), else FP8Q_ERR_SHAPE / ARG.
  * An expert id out of range sets FP8Q_ERR_DEVICE in the status word (outputs are
  * then unspecified).  Errors: NULL, ALIGN, SHAPE, ARG, CUDA. */
 fp8q_status fp8q_permute_pad_quant(const void *x, int64_t tokens, int64_t hidden, const int32_t *topk_idx,
@@ -263,8 +265,11 @@ fp8q_status fp8q_direct_transpose_mx32(const uint8_t *q, const uint8_t *sf, int6
  *   token-slot pairs with 256 experts, or 16M with 32); larger requests return
  *   FP8Q_ERR_ARG before any CUDA call.
  *   Memory: every GPU that loads the library holds the array until the process exits.
- *   Set-up: the first call on each device resolves the array's device address (with
- *   that device current); make that first call before capturing a stream.
+ *   Set-up: every call looks the array's device address up for the current device
+ *   and context (cudaGetSymbolAddress, a host-side lookup once the library's device
+ *   code is loaded), so a device reset or another context on the same device gets its
+ *   own copy's address.  The first call on a device loads that code: make it before
+ *   capturing a stream.
  *   Sharing: all calls on a device use the same array, which keeps the previous call's
  *   contents (nothing in it needs to start at zero: every word is written before it is
  *   read).  Calls that overlap on the GPU (other streams, other threads) race on it:

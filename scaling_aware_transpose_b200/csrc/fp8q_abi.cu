@@ -88,6 +88,7 @@ fp8q_status check_permute_args(const void* x, const uint8_t* xsf, bool fp8_input
                                size_t workspace_bytes) {
   if (tokens < 0 || hidden < 0 || hidden % 128 || hidden > kMaxDim) return FP8Q_ERR_SHAPE;
   if (topk < 1 || topk > 64 || num_experts < 1 || num_experts > 4096 || align < 1 || align > 4096) return FP8Q_ERR_ARG;
+  if (tokens > kMaxDim / topk) return FP8Q_ERR_SHAPE;  // row ids are int32: tokens*topk must fit
   const int64_t need = tokens * topk + (int64_t)num_experts * (align - 1);
   if (max_out_rows < need || max_out_rows > kMaxDim) return FP8Q_ERR_ARG;
   if (!expert_offsets) return FP8Q_ERR_NULL;
@@ -247,7 +248,7 @@ fp8q_status fp8q_quantize_rowwise_colwise(const void* x, int64_t rows, int64_t c
 }
 
 size_t fp8q_permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts) {
-  if (tokens < 0 || topk < 1 || num_experts < 1) return 0;
+  if (tokens < 0 || topk < 1 || num_experts < 1 || tokens > kMaxDim / topk) return 0;
   return fp8q::permute_workspace_bytes(tokens, topk, num_experts);
 }
 

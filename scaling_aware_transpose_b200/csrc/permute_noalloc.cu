@@ -12,10 +12,11 @@
 // The array is fixed-size device memory of this library: every GPU that loads the
 // library holds it until the process exits.  In host code its name is only a host-side
 // stand-in, not a device address, so the host resolves the address with
-// cudaGetSymbolAddress once per device (with that device current) and hands the pointer
-// to the kernels.
-#include <mutex>
-
+// cudaGetSymbolAddress (with the target device current) and hands the pointer to the
+// kernels.  It does so on every call: the address belongs to the module instance loaded
+// in the current context, and a device reset or a second context on the same device
+// loads another instance, so an address remembered per device could go stale.  Once the
+// module is loaded the lookup is a host-side table search.
 #include "common.cuh"
 #include "launch.h"
 
@@ -23,20 +24,12 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_permute_scratch[FP8Q_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_permute_scratch on the current device, resolved on the first call
-// for that device.  Returns nullptr if the runtime call fails.
-void* scratch_on_current_device() {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+// Device address of g_permute_scratch in the current context; nullptr if the runtime
+// call fails.
+void* scratch_in_current_context() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace
@@ -46,7 +39,9 @@ extern "C" fp8q_status fp8q_permute_pad_quant_noalloc(const void* x, int64_t tok
                                                       int32_t align, uint8_t* q, uint8_t* sf, int64_t max_out_rows,
                                                       int32_t* expert_offsets, int32_t* row_id_map,
                                                       fp8q_stream_t stream) {
-  // Size limit first, so that an oversized request fails before any CUDA call.
+  // Size limits first, so that an oversized request fails before any CUDA call; the
+  // token-slot count is bounded before anything multiplies it.
+  if (tokens > 0 && topk >= 1 && tokens > (int64_t)0x7FFFFFFF / topk) return FP8Q_ERR_SHAPE;
   if (tokens > 0 && topk >= 1 && num_experts >= 1 &&
       fp8q_permute_workspace_bytes(tokens, topk, num_experts) > (size_t)FP8Q_NOALLOC_SCRATCH_BYTES)
     return FP8Q_ERR_ARG;
@@ -56,7 +51,7 @@ extern "C" fp8q_status fp8q_permute_pad_quant_noalloc(const void* x, int64_t tok
   // totals), so nothing has to be cleared between calls.
   void* scratch = nullptr;
   if (tokens > 0) {
-    scratch = scratch_on_current_device();
+    scratch = scratch_in_current_context();
     if (scratch == nullptr) return FP8Q_ERR_CUDA;
   }
   return fp8q_permute_pad_quant(x, tokens, hidden, topk_idx, topk, num_experts, align, q, sf, max_out_rows,

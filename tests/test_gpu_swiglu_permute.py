@@ -108,32 +108,18 @@ def test_permute_zero_tokens():
 
 def test_moe_config_permute_then_grouped_transpose():
     """The MoE workload end to end: permute+pad(128)+quantize, then the grouped direct
-    transpose on the device-resident offsets; transposed output checked on every group's
-    first and last block and on a seeded sample of the rest."""
+    transpose on the device-resident offsets.  Every byte of every expert group's Q^T and
+    SF^T (all offsets[E] rows) is compared with the oracle's grouped transpose of the
+    oracle's permuted codes."""
     d = synthetic.moe()
     q, sf, off, oq, osf, ooff = check_permute(d, 32, 128)
     qt, sft = sat.direct_transpose(q, sf, off)
     device_status_ok()
     H = q.shape[1]
-    qt_h, sft_h = host(qt), host(sft)
-    rng = np.random.default_rng(0)
-    blocks = set()
-    for g in range(32):
-        a, b = int(ooff[g]), int(ooff[g + 1])
-        if a == b:
-            continue
-        blocks |= {a // 128, b // 128 - 1}
-        blocks |= set(rng.integers(a // 128, b // 128, size=4).tolist())
-    for blk in sorted(blocks):
-        g = int(np.searchsorted(ooff, blk * 128, side="right") - 1)
-        a, b = int(ooff[g]), int(ooff[g + 1])
-        M = b - a
-        r0 = blk * 128
-        want_qt, want_sft = oracle.direct_transpose(oq[r0:r0 + 128], osf[r0:r0 + 128])
-        got = qt_h[H * a: H * a + H * M].reshape(H, M)[:, r0 - a: r0 - a + 128]
-        assert_bytes_equal(got, want_qt, f"grouped Q^T block {blk}")
-        gs = sft_h[H * a // 128: H * a // 128 + H * M // 128].reshape(H, M // 128)[:, (r0 - a) // 128]
-        assert_bytes_equal(gs, want_sft[:, 0], f"grouped SF^T block {blk}")
+    n = int(ooff[-1])
+    want_qt, want_sft = oracle.direct_transpose(oq, osf, ooff)
+    assert_bytes_equal(host(sft).reshape(-1)[:H * n // 128], want_sft[:H * n // 128], "grouped SF^T")
+    assert_bytes_equal(host(qt).reshape(-1)[:H * n], want_qt[:H * n], "grouped Q^T")
 
 
 def test_bounded_wait_expires_cleanly():
