@@ -71,6 +71,8 @@ def _declare(L):
         "orc_e4m3_encode_f32_range": [ctypes.c_uint32, I64, V],
         "orc_exp_spec_f32_range": [ctypes.c_uint32, I64, V],
         "orc_direct_transpose_g": [V, V, I64, I64, I32, V, V],
+        "orc_ep_dispatch_pack": [V, V, I64, I64, V, I32, I32, I32, V, V, V, I64, V, V],
+        "orc_ep_recv_permute": [V, V, V, I64, I64, I32, I32, I32, V, V, I64, V, V],
     }.items():
         fn = getattr(L, name)
         fn.argtypes, fn.restype = args, ctypes.c_int
@@ -314,6 +316,55 @@ def permute_pad_fp8(q_bits, sf, topk_idx, num_experts: int, align: int, max_rows
                                    _p(off), _p(rmap))
     if rc:
         raise OracleError(f"oracle FP8 permute rejected its arguments (code {rc})")
+    return q, osf, off, rmap
+
+
+def ep_dispatch_pack(q_bits, sf, topk_idx, num_ranks: int, experts_per_rank: int, fill: int = 0xEE):
+    """Send side of one source rank of the expert-parallel FP8 dispatch: returns
+    (send_q [S, H], send_sf [S, H/128], send_ids [S, K], send_offsets [W+1],
+    send_map [T, W]) with S = send_offsets[W] (every token sent once to each rank that
+    holds one of its experts, grouped by destination rank)."""
+    xq = _c(q_bits, np.uint8)
+    xsf = _c(sf, np.uint8)
+    idx = _c(topk_idx, np.int32)
+    T, H = xq.shape
+    K = idx.shape[1]
+    W = num_ranks
+    cap = T * W
+    sq = np.full((cap, H), fill, np.uint8)
+    ssf = np.full((cap, H // 128), fill, np.uint8)
+    sids = np.full((cap, K), -7, np.int32)
+    soff = np.zeros(W + 1, np.int32)
+    smap = np.zeros((T, W), np.int32)
+    rc = lib().orc_ep_dispatch_pack(_p(xq), _p(xsf), T, H, _p(idx), K, W, experts_per_rank, _p(sq), _p(ssf),
+                                    _p(sids), cap, _p(soff), _p(smap))
+    if rc:
+        raise OracleError(f"oracle EP dispatch pack rejected its arguments (code {rc})")
+    S = int(soff[W])
+    return sq[:S], ssf[:S], sids[:S], soff, smap
+
+
+def ep_recv_permute(recv_q, recv_sf, recv_ids, experts_per_rank: int, align: int, max_rows: int | None = None,
+                    fill: int = 0xEE):
+    """Receive side of one destination rank: the rows received from every source rank
+    (concatenated in source-rank order) -> (Q [max_rows, H], SF [max_rows, H/128],
+    offsets [Eloc+1], row_id_map [R*K]); slots with id -1 (expert on another rank)
+    get row id -1."""
+    rq = _c(recv_q, np.uint8)
+    rsf = _c(recv_sf, np.uint8)
+    rids = _c(recv_ids, np.int32)
+    R, H = rq.shape
+    K = rids.shape[1] if rids.ndim == 2 else 1
+    if max_rows is None:
+        max_rows = permute_max_rows(R, K, experts_per_rank, align)
+    q = np.full((max_rows, H), fill, np.uint8)
+    osf = np.full((max_rows, H // 128), fill, np.uint8)
+    off = np.zeros(experts_per_rank + 1, np.int32)
+    rmap = np.zeros(R * K, np.int32)
+    rc = lib().orc_ep_recv_permute(_p(rq), _p(rsf), _p(rids), R, H, K, experts_per_rank, align, _p(q), _p(osf),
+                                   max_rows, _p(off), _p(rmap))
+    if rc:
+        raise OracleError(f"oracle EP receive permute rejected its arguments (code {rc})")
     return q, osf, off, rmap
 
 

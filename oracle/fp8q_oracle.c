@@ -785,6 +785,131 @@ int orc_permute_pad_fp8(const uint8_t *xq, const uint8_t *xsf, int64_t T, int64_
 }
 
 /* ------------------------------------------------------------------ */
+/* Expert-parallel FP8 dispatch ([FLOW] 核心方法: the dispatch carries   */
+/* row-wise FP8 codes with their scale metadata, Table 1: FP8 all-to-all */
+/* beats BF16; [DSV3] §5.6: each rank's experts read contiguous rows)    */
+/* ------------------------------------------------------------------ */
+
+/* Send side of one source rank.  Experts are numbered globally, expert e living on
+ * rank e / Eloc as its local expert e % Eloc (W ranks, Eloc experts each).  A token is
+ * sent once to every rank that holds at least one of its K experts (its destination
+ * set), carrying its row-wise codes, its scale bytes and its K slot ids re-expressed
+ * for that rank: the local expert id where the slot's expert lives there, -1 where it
+ * lives elsewhere.  The send buffer is grouped by destination rank, tokens in order
+ * within a group: send_offsets[d] = number of rows for ranks below d, and the row of
+ * (token t, rank d) is send_offsets[d] + (number of tokens before t sent to d);
+ * send_map[t*W + d] holds it, or -1 where t is not sent to d.
+ * Returns 2 on bad sizes, 7 on an expert id outside [0, W*Eloc), 4 when the rows
+ * exceed max_rows. */
+int orc_ep_dispatch_pack(const uint8_t *xq, const uint8_t *xsf, int64_t T, int64_t H, const int32_t *idx,
+                         int32_t K, int32_t W, int32_t Eloc, uint8_t *send_q, uint8_t *send_sf, int32_t *send_ids,
+                         int64_t max_rows, int32_t *send_offsets, int32_t *send_map)
+{
+    if (H % 128 || T < 0 || K < 1 || W < 1 || Eloc < 1)
+        return 2;
+    int64_t nt = H / 128;
+    for (int64_t p = 0; p < T * K; p++)
+        if (idx[p] < 0 || idx[p] >= (int64_t)W * Eloc)
+            return 7;
+    int64_t *cnt = (int64_t *)calloc((size_t)W, sizeof(int64_t));
+    if (!cnt)
+        return 5;
+    /* destination set of each token, counted per rank */
+    for (int64_t t = 0; t < T; t++)
+        for (int32_t d = 0; d < W; d++) {
+            int hit = 0;
+            for (int32_t k = 0; k < K; k++)
+                hit |= idx[t * K + k] / Eloc == d;
+            send_map[t * W + d] = hit ? 0 : -1;
+            cnt[d] += hit;
+        }
+    int64_t acc = 0;
+    for (int32_t d = 0; d < W; d++) {
+        send_offsets[d] = (int32_t)acc;
+        acc += cnt[d];
+    }
+    send_offsets[W] = (int32_t)acc;
+    if (acc > max_rows) {
+        free(cnt);
+        return 4;
+    }
+    memset(cnt, 0, (size_t)W * sizeof(int64_t));
+    for (int64_t t = 0; t < T; t++)
+        for (int32_t d = 0; d < W; d++) {
+            if (send_map[t * W + d] < 0)
+                continue;
+            int64_t r = send_offsets[d] + cnt[d]++;
+            send_map[t * W + d] = (int32_t)r;
+            memcpy(send_q + r * H, xq + t * H, (size_t)H);
+            memcpy(send_sf + r * nt, xsf + t * nt, (size_t)nt);
+            for (int32_t k = 0; k < K; k++) {
+                int32_t e = idx[t * K + k];
+                send_ids[r * K + k] = e / Eloc == d ? e - d * Eloc : -1;
+            }
+        }
+    free(cnt);
+    return 0;
+}
+
+/* Receive side of one destination rank: the rows received from all source ranks,
+ * concatenated in source-rank order (rank 0's rows first, each source's rows in its
+ * send order), with their slot ids (local expert ids, -1 for slots whose expert lives
+ * on another rank).  Slot (r, s) with id e >= 0 goes to local expert e; the rows of an
+ * expert follow (r, s) row-major order and each expert's segment is padded with zero
+ * rows (codes 0x00, scale byte 127) to a multiple of align, exactly as the FP8-input
+ * permute does; a slot with id -1 gets row_id_map -1 and no row.
+ * Returns 2 on bad sizes, 7 on an id outside [-1, Eloc), 4 when rows exceed max_rows. */
+int orc_ep_recv_permute(const uint8_t *rq, const uint8_t *rsf, const int32_t *rids, int64_t R, int64_t H, int32_t K,
+                        int32_t Eloc, int32_t align, uint8_t *q, uint8_t *sf, int64_t max_rows, int32_t *offsets,
+                        int32_t *row_id_map)
+{
+    if (H % 128 || R < 0 || K < 1 || Eloc < 1 || align < 1)
+        return 2;
+    int64_t nt = H / 128;
+    int64_t *cnt = (int64_t *)calloc((size_t)Eloc, sizeof(int64_t));
+    if (!cnt)
+        return 5;
+    for (int64_t p = 0; p < R * K; p++) {
+        if (rids[p] < -1 || rids[p] >= Eloc) {
+            free(cnt);
+            return 7;
+        }
+        if (rids[p] >= 0)
+            cnt[rids[p]]++;
+    }
+    int64_t acc = 0;
+    for (int32_t e = 0; e < Eloc; e++) {
+        offsets[e] = (int32_t)acc;
+        acc += (cnt[e] + align - 1) / align * align;
+    }
+    offsets[Eloc] = (int32_t)acc;
+    if (acc > max_rows) {
+        free(cnt);
+        return 4;
+    }
+    int64_t *seen = cnt;
+    memset(seen, 0, (size_t)Eloc * sizeof(int64_t));
+    for (int64_t p = 0; p < R * K; p++) {
+        int32_t e = rids[p];
+        if (e < 0) {
+            row_id_map[p] = -1;
+            continue;
+        }
+        int64_t r = offsets[e] + seen[e]++;
+        row_id_map[p] = (int32_t)r;
+        memcpy(q + r * H, rq + (p / K) * H, (size_t)H);
+        memcpy(sf + r * nt, rsf + (p / K) * nt, (size_t)nt);
+    }
+    for (int32_t e = 0; e < Eloc; e++)
+        for (int64_t r = offsets[e] + seen[e]; r < offsets[e + 1]; r++) {
+            memset(q + r * H, 0x00, (size_t)H);
+            memset(sf + r * nt, 127, (size_t)nt);
+        }
+    free(cnt);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Fused unpermute + unpad ([FLOW] 核心方法: Fused Permute+Padding /    */
 /* Unpermute+Unpadding; the combine side of the expert path)           */
 /* ------------------------------------------------------------------ */
