@@ -32,6 +32,13 @@ class Fp8qError(RuntimeError):
         super().__init__(f"{where}: {STATUS.get(self.status, self.status)} ({_status_string(self.status)})")
 
 
+class EpSource(ctypes.Structure):
+    """fp8q_ep_source: one received segment (device pointers and its row count)."""
+    _fields_ = [("q", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("ids", ctypes.c_void_p), ("rows", ctypes.c_int64)]
+
+
+EP_MAX_RANKS = 64  # FP8Q_EP_MAX_RANKS
+
 _lib = None
 
 
@@ -66,6 +73,11 @@ def lib() -> ctypes.CDLL:
             "fp8q_debug_exp_spec_range": ([ctypes.c_uint32, I64, P, P], ctypes.c_int),
             "fp8q_debug_swiglu_spec": ([P, P, I64, P, P], ctypes.c_int),
             "fp8q_debug_silu_bf16": ([P, I64, P, P], ctypes.c_int),
+            "fp8q_ep_pack_workspace_bytes": ([I64, I32], SZ),
+            "fp8q_ep_dispatch_pack": ([P, P, I64, I64, P, I32, I32, I32, P, P, P, I64, P, P, P, SZ, P], ctypes.c_int),
+            "fp8q_ep_recv_workspace_bytes": ([I64, I32, I32], SZ),
+            "fp8q_ep_recv_permute_fp8": ([ctypes.POINTER(EpSource), I32, I64, I32, I32, I32, P, P, I64, P, P, P, SZ,
+                                          P], ctypes.c_int),
             "fp8q_version": ([], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -386,3 +398,74 @@ def direct_transpose_mx32(q, sf, stream=None):
     sft = _empty((cols, rows // 32), torch.uint8, q)
     fp8q_direct_transpose_mx32(q, sf, rows, cols, qt, sft, stream)
     return qt, sft
+
+
+# ---------------------------------------------------------------- expert-parallel dispatch
+def fp8q_ep_pack_workspace_bytes(tokens: int, num_ranks: int) -> int:
+    return int(lib().fp8q_ep_pack_workspace_bytes(tokens, num_ranks))
+
+
+def fp8q_ep_recv_workspace_bytes(rows: int, topk: int, experts_per_rank: int) -> int:
+    return int(lib().fp8q_ep_recv_workspace_bytes(rows, topk, experts_per_rank))
+
+
+def fp8q_ep_dispatch_pack(xq, xsf, tokens: int, hidden: int, topk_idx, topk: int, num_ranks: int,
+                          experts_per_rank: int, send_q, send_sf, send_ids, max_send_rows: int, send_offsets,
+                          send_map, workspace, workspace_bytes: int, stream=None) -> None:
+    _check(lib().fp8q_ep_dispatch_pack(_ptr(xq), _ptr(xsf), tokens, hidden, _ptr(topk_idx), topk, num_ranks,
+                                       experts_per_rank, _ptr(send_q), _ptr(send_sf), _ptr(send_ids), max_send_rows,
+                                       _ptr(send_offsets), _ptr(send_map), _ptr(workspace), workspace_bytes,
+                                       _stream(stream)), "fp8q_ep_dispatch_pack")
+
+
+def fp8q_ep_recv_permute_fp8(segments, hidden: int, topk: int, experts_per_rank: int, align: int, q, sf,
+                             max_out_rows: int, expert_offsets, row_id_map, workspace, workspace_bytes: int,
+                             stream=None) -> None:
+    """segments: sequence of (q, sf, ids, rows) with q/sf/ids device tensors (or raw
+    device addresses as ints) of the received rows of one source rank each."""
+    arr = (EpSource * len(segments))()
+    for i, (sq, ssf, sids, rows) in enumerate(segments):
+        arr[i] = EpSource(_ptr(sq), _ptr(ssf), _ptr(sids), int(rows))
+    _check(lib().fp8q_ep_recv_permute_fp8(arr, len(segments), hidden, topk, experts_per_rank, align, _ptr(q), _ptr(sf),
+                                          max_out_rows, _ptr(expert_offsets), _ptr(row_id_map), _ptr(workspace),
+                                          workspace_bytes, _stream(stream)), "fp8q_ep_recv_permute_fp8")
+
+
+def ep_dispatch_pack(xq, xsf, topk_idx, num_ranks: int, experts_per_rank: int, stream=None):
+    """Send side of one rank: (send_q [cap, H], send_sf [cap, H/128], send_ids [cap, K],
+    send_offsets [W+1], send_map [T, W]); rows send_offsets[W] and beyond are unused."""
+    import torch
+    tokens, hidden = xq.shape
+    topk = topk_idx.shape[1]
+    cap = max(tokens * min(num_ranks, topk), 1)
+    send_q = _empty((cap, hidden), torch.uint8, xq)
+    send_sf = _empty((cap, hidden // 128), torch.uint8, xq)
+    send_ids = _empty((cap, topk), torch.int32, xq)
+    send_off = _empty((num_ranks + 1,), torch.int32, xq)
+    send_map = _empty((tokens, num_ranks), torch.int32, xq)
+    ws_bytes = fp8q_ep_pack_workspace_bytes(tokens, num_ranks)
+    ws = _empty((max(ws_bytes, 16),), torch.uint8, xq)
+    fp8q_ep_dispatch_pack(xq, xsf, tokens, hidden, topk_idx, topk, num_ranks, experts_per_rank, send_q, send_sf,
+                          send_ids, cap, send_off, send_map, ws, ws.numel(), stream)
+    return send_q, send_sf, send_ids, send_off, send_map
+
+
+def ep_recv_permute(segments, experts_per_rank: int, align: int, max_out_rows: int | None = None, stream=None):
+    """Receive side of one rank from per-source segments (q [n, H], sf [n, H/128],
+    ids [n, K]) -> (q [max_out_rows, H], sf, expert_offsets [Eloc+1], row_id_map [R*K])."""
+    import torch
+    ref = next(s[0] for s in segments)
+    hidden = ref.shape[1]
+    topk = next(s[2] for s in segments).shape[1]
+    rows = sum(int(s[0].shape[0]) for s in segments)
+    if max_out_rows is None:
+        max_out_rows = permute_max_rows(rows, topk, experts_per_rank, align)
+    q = _empty((max(max_out_rows, 1), hidden), torch.uint8, ref)
+    sf = _empty((max(max_out_rows, 1), hidden // 128), torch.uint8, ref)
+    off = _empty((experts_per_rank + 1,), torch.int32, ref)
+    rmap = _empty((max(rows * topk, 1),), torch.int32, ref)
+    ws_bytes = fp8q_ep_recv_workspace_bytes(rows, topk, experts_per_rank)
+    ws = _empty((max(ws_bytes, 16),), torch.uint8, ref)
+    fp8q_ep_recv_permute_fp8([(a, b, c, a.shape[0]) for a, b, c in segments], hidden, topk, experts_per_rank, align,
+                             q, sf, max_out_rows, off, rmap, ws, ws.numel(), stream)
+    return q, sf, off, rmap[:rows * topk]

@@ -41,6 +41,20 @@ fp8q_status launch_quantize_rowwise_colwise(const DeviceInfo& dev, const void* x
                                             cudaStream_t stream);
 
 size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts);
+// Routing of rows x slots pairs (idx [rows, slots], ids in [0, E)) to E groups: counts,
+// offsets of the groups padded to `align`, stable (row, slot) row ids.  With allow_drop
+// an id of -1 gives row id -1 and no row.  workspace >= permute_workspace_bytes(rows,
+// slots, E); route_totals() points at the per-group pair counts inside it.
+fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx, int32_t slots, int32_t E,
+                        int32_t align, bool allow_drop, int32_t* offsets, int32_t* row_id_map, void* workspace,
+                        cudaStream_t stream);
+const int32_t* route_totals(const void* workspace, int64_t rows, int32_t slots, int32_t E);
+// FP8 payload of a routing: row r's codes and scale bytes go to rows row_id_map[r*slots
+// + s] (skipped where -1); the trailing CTAs zero-fill each group's padding rows.  A
+// programmatic dependent launch: it waits for the routing kernels before reading ids.
+fp8q_status launch_scatter_copy(const uint8_t* xq, const uint8_t* xsf, int64_t rows, int64_t hidden,
+                                const int32_t* row_id_map, int32_t slots, int32_t E, int32_t align, uint8_t* q,
+                                uint8_t* sf, const int32_t* offsets, const int32_t* totals, cudaStream_t stream);
 fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,
                                      const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
                                      uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,

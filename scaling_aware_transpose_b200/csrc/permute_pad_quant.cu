@@ -17,29 +17,16 @@
 // The FP8-input variant (the dispatch already delivered row-wise codes and scales) shares
 // (1)-(3) and the padding; its step (4) copies each token's codes and scale bytes to its
 // rows.
-#include "common.cuh"
 #include "launch.h"
+#include "permute_common.cuh"
 
 namespace fp8q {
 namespace {
 
-constexpr int kChunk = 1024;  // (t, s) pairs per chunk, in row-major order
-
-// Programmatic dependent launch (sm_90 and later): the scan, rank and scatter launches
-// carry the programmatic-stream-serialization attribute, so each may be scheduled while
-// its predecessor in the chain still runs.  pdl_wait() returns once the predecessor grid
-// has completed and its writes are visible (a hardware dependency, not a spin loop);
-// pdl_trigger() lets the successor be scheduled.  In a launch without the attribute both
-// are no-ops.  The first kernel of a call (the histogram) is launched plainly, so no part
-// of a call overlaps work queued before it.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-constexpr int kMaxExperts = 4096;
-
-int64_t num_chunks(int64_t tokens, int32_t topk) { return (tokens * topk + kChunk - 1) / kChunk; }
-
+// allow_drop: an id of -1 means "not routed here" (no row, no error); any other id
+// outside [0, E) records FP8Q_ERR_DEVICE.
 __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
-                                                    int32_t* __restrict__ counts, int* status) {
+                                                    bool allow_drop, int32_t* __restrict__ counts, int* status) {
   extern __shared__ int32_t hist[];
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
@@ -50,7 +37,7 @@ __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ 
     if (p >= npairs) break;
     const int32_t e = __ldg(idx + p);
     if (e < 0 || e >= E) {
-      record_status(status, FP8Q_ERR_DEVICE);
+      if (!(allow_drop && e == -1)) record_status(status, FP8Q_ERR_DEVICE);
       continue;
     }
     atomicAdd(&hist[e], 1);
@@ -246,29 +233,6 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
   }
 }
 
-// Padding rows: CTA slot `slot` of expert e zeroes rows offsets[e] + totals[e] + 8*slot ..
-// (at most 8 rows, never past offsets[e+1]): codes 0x00, scale byte 127.  Run by the
-// trailing CTAs of the scatter launch (E x ceil((align-1)/8) of them).
-constexpr int kPadRowsPerCta = 8;
-__device__ __forceinline__ void pad_rows(int64_t pad_cta, int pad_slots, const int32_t* __restrict__ offsets,
-                                         const int32_t* __restrict__ totals, int64_t hidden, uint8_t* __restrict__ q,
-                                         uint8_t* __restrict__ sf) {
-  const int e = (int)(pad_cta / pad_slots);
-  const int slot = (int)(pad_cta - (int64_t)e * pad_slots);
-  const int64_t start = (int64_t)offsets[e] + totals[e], end = offsets[e + 1];
-  const int64_t ncb = hidden >> 7;
-  for (int rr = 0; rr < kPadRowsPerCta; ++rr) {
-    const int64_t r = start + (int64_t)slot * kPadRowsPerCta + rr;
-    if (r >= end) return;
-    uint4* row = reinterpret_cast<uint4*>(q + r * hidden);
-    for (int64_t i = threadIdx.x; i < hidden / 16; i += blockDim.x) row[i] = make_uint4(0u, 0u, 0u, 0u);
-    for (int64_t i = threadIdx.x; i < ncb; i += blockDim.x) sf[r * ncb + i] = 127;
-  }
-}
-
-constexpr int kSThreads = 256;
-constexpr int kSUnroll = 2;
-
 // Tiles of x (token t, column block j) in row-major order: 8 lanes per tile, 16 bf16 per
 // lane (8 from each half of the tile), four tiles per warp per slot.  Each tile is read
 // and quantized once and its codes written to the token's top-k destination rows.
@@ -385,45 +349,35 @@ size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts
   return (size_t)(2 * C * num_experts + num_experts) * sizeof(int32_t) + 16;
 }
 
-namespace {
-
-// A launch that may begin while the previous kernel in the stream finishes (see pdl_wait).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_after(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
-                         Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
-// Steps (1)-(3): offsets, per-chunk bases, row ids.
-fp8q_status route(const DeviceInfo& dev, int64_t tokens, const int32_t* topk_idx, int32_t topk, int E, int32_t align,
-                  int32_t* expert_offsets, int32_t* row_id_map, int32_t* counts, int32_t* bases, int32_t* totals,
-                  cudaStream_t stream) {
-  const int64_t npairs = tokens * topk;
-  const int64_t C = num_chunks(tokens, topk);
+// Steps (1)-(3): offsets, per-chunk bases, row ids (workspace: counts, bases, totals).
+fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx, int32_t slots, int32_t E,
+                        int32_t align, bool allow_drop, int32_t* offsets, int32_t* row_id_map, void* workspace,
+                        cudaStream_t stream) {
+  const int64_t npairs = rows * slots;
+  const int64_t C = num_chunks(rows, slots);
+  int32_t* counts = static_cast<int32_t*>(workspace);
+  int32_t* bases = counts + C * E;
+  int32_t* totals = bases + C * E;
   const size_t hist_smem = (size_t)E * sizeof(int32_t);
-  count_kernel<<<(unsigned)C, 256, hist_smem, stream>>>(topk_idx, npairs, E, counts, dev.status);
+  count_kernel<<<(unsigned)C, 256, hist_smem, stream>>>(idx, npairs, E, allow_drop, counts, dev.status);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  if (launch_after(scan_kernel, 1, 1024, 0, stream, (const int32_t*)counts, C, E, (int)align, expert_offsets, bases,
+  if (launch_after(scan_kernel, 1, 1024, 0, stream, (const int32_t*)counts, C, E, (int)align, offsets, bases,
                    totals) != cudaSuccess)
     return FP8Q_ERR_CUDA;
   const cudaError_t rc =
       E <= kRankMultiMaxE
           ? launch_after(rank_multi_kernel, (unsigned)C, kRankWarps * 32, (size_t)kRankWarps * E * sizeof(int32_t),
-                         stream, topk_idx, npairs, E, (const int32_t*)bases, row_id_map)
-          : launch_after(rank_kernel, (unsigned)C, 32, hist_smem, stream, topk_idx, npairs, E, (const int32_t*)bases,
+                         stream, idx, npairs, E, (const int32_t*)bases, row_id_map)
+          : launch_after(rank_kernel, (unsigned)C, 32, hist_smem, stream, idx, npairs, E, (const int32_t*)bases,
                          row_id_map);
   return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
+
+const int32_t* route_totals(const void* workspace, int64_t rows, int32_t slots, int32_t E) {
+  return static_cast<const int32_t*>(workspace) + 2 * num_chunks(rows, slots) * E;
+}
+
+namespace {
 
 // xq/xsf != nullptr: FP8-input payload; else quantize x.
 fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq, const uint8_t* xsf, int64_t tokens,
@@ -436,13 +390,10 @@ fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq,
                ? FP8Q_OK
                : FP8Q_ERR_CUDA;
   }
-  const int64_t C = num_chunks(tokens, topk);
-  int32_t* counts = static_cast<int32_t*>(workspace);
-  int32_t* bases = counts + C * E;
-  int32_t* totals = bases + C * E;
-  const fp8q_status rs = route(dev, tokens, topk_idx, topk, E, align, expert_offsets, row_id_map, counts, bases,
-                               totals, stream);
+  const fp8q_status rs =
+      route_pairs(dev, tokens, topk_idx, topk, E, align, false, expert_offsets, row_id_map, workspace, stream);
   if (rs != FP8Q_OK) return rs;
+  const int32_t* totals = route_totals(workspace, tokens, topk, E);
   if (hidden == 0) return FP8Q_OK;  // routing only: offsets and row ids, no payload
   const int ncb = (int)(hidden / 128);
   const int64_t n_tiles = tokens * ncb;
@@ -454,17 +405,30 @@ fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq,
   const int32_t* rmap = row_id_map;
   const int32_t* offs = expert_offsets;
   const int32_t* tots = totals;
-  const cudaError_t rc =
-      xq ? launch_after(scatter_copy_kernel, (unsigned)blocks, kSThreads, 0, stream,
-                        reinterpret_cast<const uint4*>(xq), xsf, tokens, ncb, rmap, (int)topk,
-                        reinterpret_cast<uint4*>(q), sf, scatter_ctas, pad_slots, offs, tots)
-         : launch_after(scatter_quant_kernel, (unsigned)blocks, kSThreads, 0, stream, static_cast<const uint4*>(x),
-                        tokens, ncb, rmap, (int)topk, reinterpret_cast<uint2*>(q), sf, scatter_ctas, pad_slots, offs,
-                        tots);
+  if (xq) return launch_scatter_copy(xq, xsf, tokens, hidden, rmap, topk, E, align, q, sf, offs, tots, stream);
+  const cudaError_t rc = launch_after(scatter_quant_kernel, (unsigned)blocks, kSThreads, 0, stream,
+                                      static_cast<const uint4*>(x), tokens, ncb, rmap, (int)topk,
+                                      reinterpret_cast<uint2*>(q), sf, scatter_ctas, pad_slots, offs, tots);
   return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 }  // namespace
+
+fp8q_status launch_scatter_copy(const uint8_t* xq, const uint8_t* xsf, int64_t rows, int64_t hidden,
+                                const int32_t* row_id_map, int32_t slots, int32_t E, int32_t align, uint8_t* q,
+                                uint8_t* sf, const int32_t* offsets, const int32_t* totals, cudaStream_t stream) {
+  const int ncb = (int)(hidden / 128);
+  const int64_t n_tiles = rows * ncb;
+  const int64_t tiles_per_block = (kSThreads / 32) * kSUnroll * 4;
+  const int64_t scatter_ctas = (n_tiles + tiles_per_block - 1) / tiles_per_block;
+  const int pad_slots = (align - 1 + kPadRowsPerCta - 1) / kPadRowsPerCta;  // 0 when align == 1
+  const int64_t blocks = scatter_ctas + (int64_t)E * pad_slots;
+  if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const cudaError_t rc = launch_after(scatter_copy_kernel, (unsigned)blocks, kSThreads, 0, stream,
+                                      reinterpret_cast<const uint4*>(xq), xsf, rows, ncb, row_id_map, (int)slots,
+                                      reinterpret_cast<uint4*>(q), sf, scatter_ctas, pad_slots, offsets, totals);
+  return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
 
 fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,
                                      const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,

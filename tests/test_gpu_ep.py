@@ -1,0 +1,135 @@
+"""GPU parity of the expert-parallel FP8 dispatch against the CPU oracle, byte for byte.
+
+W ranks are simulated on one GPU: each source rank's tokens are packed by
+fp8q_ep_dispatch_pack; each destination rank's receive permute (fp8q_ep_recv_permute_fp8)
+is then given, as its segments, the slices of the source ranks' send buffers that an
+all-to-all would deliver to it - read in place, as they would be read from a receive
+buffer.  The exchange itself runs through NCCL on a one-rank group (all this machine
+offers); its multi-rank logic is covered on gloo ranks in test_ep_host.py.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scaling_aware_transpose_b200 as sat
+from scaling_aware_transpose_b200 import synthetic
+from gpu_helpers import assert_bytes_equal, dev, device_status_ok, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _sources(W, T, H, K, Eloc, seed, row_sigma=1.0):
+    rng = np.random.default_rng(seed)
+    xs, idx = [], []
+    for s in range(W):
+        q, sf = oracle.quantize_rowwise(synthetic.scaled_normal(T, H, seed=seed + s, row_sigma=row_sigma))
+        xs.append((q, sf))
+        idx.append(synthetic.zipf_topk(T, W * Eloc, K, rng) if T else np.zeros((0, K), np.int32))
+    return xs, idx
+
+
+def _check_pack(got, want, T):
+    sq, ssf, sids, soff, smap = got
+    oq, osf, oids, ooff, omap = want
+    assert_bytes_equal(host(soff), ooff, "send offsets")
+    assert_bytes_equal(host(smap), omap, "send map")
+    S = int(ooff[-1])
+    assert_bytes_equal(host(sids)[:S], oids, "send ids")
+    assert_bytes_equal(host(ssf)[:S], osf, "send SF")
+    assert_bytes_equal(host(sq)[:S], oq, "send Q")
+
+
+def run_ep(W, T, H, K, Eloc, align, seed=0):
+    """Pack on every simulated source rank, receive-permute on every destination rank;
+    compare each step with the oracle and the result with the global FP8 permute."""
+    xs, idx = _sources(W, T, H, K, Eloc, seed)
+    packs_d, packs_o = [], []
+    for s in range(W):
+        got = sat.ep_dispatch_pack(dev(xs[s][0]), dev(xs[s][1]), dev(idx[s]), W, Eloc)
+        device_status_ok()
+        want = oracle.ep_dispatch_pack(xs[s][0], xs[s][1], idx[s], W, Eloc)
+        _check_pack(got, want, T)
+        packs_d.append(got)
+        packs_o.append(want)
+    gq, gsf, goff, _ = oracle.permute_pad_fp8(np.concatenate([x[0] for x in xs]), np.concatenate([x[1] for x in xs]),
+                                              np.concatenate(idx), W * Eloc, align)
+    for d in range(W):
+        segs = []
+        for s in range(W):
+            a, b = int(packs_o[s][3][d]), int(packs_o[s][3][d + 1])
+            sq, ssf, sids = packs_d[s][0], packs_d[s][1], packs_d[s][2]
+            segs.append((sq[a:b], ssf[a:b], sids[a:b]))
+        q, sf, off, rmap = sat.ep_recv_permute(segs, Eloc, align)
+        device_status_ok()
+        rq = np.concatenate([p[0][p[3][d]:p[3][d + 1]] for p in packs_o])
+        rsf = np.concatenate([p[1][p[3][d]:p[3][d + 1]] for p in packs_o])
+        rids = np.concatenate([p[2][p[3][d]:p[3][d + 1]] for p in packs_o])
+        oq, osf, ooff, ormap = oracle.ep_recv_permute(rq, rsf, rids, Eloc, align)
+        assert_bytes_equal(host(off), ooff, f"rank {d} expert offsets")
+        assert_bytes_equal(host(rmap), ormap, f"rank {d} row_id_map")
+        n = int(ooff[-1])
+        assert_bytes_equal(host(sf)[:n], osf[:n], f"rank {d} SF")
+        assert_bytes_equal(host(q)[:n], oq[:n], f"rank {d} Q")
+        base = int(goff[d * Eloc])
+        assert np.array_equal(oq[:n], gq[base:base + n])
+
+
+@pytest.mark.parametrize("W,T,H,K,Eloc,align", [(2, 300, 256, 4, 4, 16), (4, 512, 384, 8, 8, 128),
+                                                 (8, 200, 128, 2, 1, 1), (3, 1000, 512, 6, 5, 64),
+                                                 (1, 700, 256, 3, 7, 16), (5, 0, 256, 2, 2, 16)])
+def test_ep_dispatch_simulated_ranks(W, T, H, K, Eloc, align):
+    run_ep(W, T, H, K, Eloc, align, seed=W * 7 + T)
+
+
+def test_ep_dispatch_moe_workload():
+    """The MoE workload split over 4 expert-parallel ranks: 4 x 4096 tokens of hidden 7168,
+    top-8 of 32 Zipf(1.1) experts, 8 experts per rank, 128-row alignment."""
+    run_ep(4, 4096, 7168, 8, 8, 128, seed=0)
+
+
+def test_ep_many_ranks_and_empty_segments():
+    """64 ranks (the maximum), one expert each, few tokens: many empty segments."""
+    run_ep(64, 20, 128, 2, 1, 16, seed=3)
+
+
+def test_ep_bad_ids_set_device_status():
+    q = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
+    sf = torch.full((4, 1), 127, dtype=torch.uint8, device="cuda")
+    idx = torch.tensor([[0], [1], [9], [2]], dtype=torch.int32, device="cuda")
+    sat.ep_dispatch_pack(q, sf, idx, 2, 4)
+    assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE
+    ids = torch.tensor([[0], [-2], [1], [2]], dtype=torch.int32, device="cuda")
+    sat.ep_recv_permute([(q, sf, ids)], 4, 16)
+    assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE
+
+
+def test_ep_dispatch_through_nccl_one_rank():
+    """ep.dispatch end to end over a one-rank NCCL group: all_to_all_single of device
+    buffers, then the receive permute; with one rank the result is the FP8 permute's."""
+    import torch.distributed as dist
+    from scaling_aware_transpose_b200 import ep
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0),
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        xs, idx = _sources(1, 2048, 1024, 8, 16, seed=5)
+        res = ep.dispatch(dev(xs[0][0]), dev(xs[0][1]), dev(idx[0]), 16, 128)
+        device_status_ok()
+        oq, osf, ooff, ormap = oracle.permute_pad_fp8(xs[0][0], xs[0][1], idx[0], 16, 128)
+        assert_bytes_equal(host(res.expert_offsets), ooff, "offsets")
+        assert_bytes_equal(host(res.row_id_map), ormap, "row_id_map")
+        n = int(ooff[-1])
+        assert_bytes_equal(host(res.q)[:n], oq[:n], "Q")
+        assert_bytes_equal(host(res.sf)[:n], osf[:n], "SF")
+        assert res.recv_counts == res.send_counts == [2048]
+    finally:
+        dist.destroy_process_group()
