@@ -241,7 +241,8 @@ fp8q_status fp8q_permute_pad_fp8(const uint8_t *xq, const uint8_t *xsf, int64_t 
  *   fp8q_direct_transpose_mx32: (q, sf) as above -> qt u8 [cols, rows], sft u8
  *     [cols, rows/32] holding, for channel h and token group g, the largest scale byte of
  *     the 32x32 block (g, h/32).  This build's kernel needs rows % 128 == 0 and
- *     cols % 128 == 0 (its CTA tile is 128x128, sixteen MX blocks).  q and qt 16-byte
+ *     cols % 128 == 0 (its CTA tile is 128x128, sixteen MX blocks), and rows at most
+ *     65535 * 128 (its grid has one row of CTAs per 128 rows).  q and qt 16-byte
  *     aligned, sf and sft 4-byte aligned.
  * Errors: NULL, ALIGN, SHAPE, CUDA. */
 fp8q_status fp8q_quantize_rowwise_mx32(const void *x, int64_t rows, int64_t cols, uint8_t *q, uint8_t *sf,

@@ -145,10 +145,12 @@ __device__ __forceinline__ uint32_t shift_word_general(uint32_t w, uint32_t s2) 
       : "r"(w), "r"(s2));
   return r;
 }
-// One 16-byte row chunk: the SWAR subtract when it is exact for every byte, else the
-// general form (per-lane branch; used where rows rarely need re-rounding).
-__device__ __forceinline__ void shift_row16(uint32_t (&w)[4], int k) {
-  if (shift_fast_ok(w, k)) {
+// One 16-byte row chunk per lane, the form chosen once per warp: the SWAR subtract when
+// it is exact for every lane's 16 bytes, else the general form on every lane.  A per-lane choice
+// makes a warp that mixes the two run both; on real activations most warps hold some
+// lane that needs the general form.  Every lane of the warp must call it.
+__device__ __forceinline__ void shift_row16_warp(uint32_t (&w)[4], int k) {
+  if (__all_sync(0xFFFFFFFFu, shift_fast_ok(w, k))) {
     const uint32_t kk = (uint32_t)k * 0x08080808u;
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] -= kk;
@@ -247,5 +249,9 @@ __device__ __forceinline__ int64_t grouped_rows(const int32_t* off, int G, int64
 
 // ------------------------------------------------------------------ memory
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
+// 8-byte store marked evict-first (written once, not read again by this kernel).
+__device__ __forceinline__ void st_stream8(void* p, uint2 v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
 
 }  // namespace fp8q

@@ -72,10 +72,13 @@ __global__ void __launch_bounds__(256) dest_kernel(const int32_t* __restrict__ i
   didx[p] = hit ? d : -1;
 }
 
-// Slot ids of each sent row, re-expressed for its destination rank.
+// Slot ids of each sent row, re-expressed for its destination rank.  A dependent launch
+// after the routing: it waits for the send map before reading it.
 __global__ void __launch_bounds__(256) send_ids_kernel(const int32_t* __restrict__ idx, int64_t tokens, int K, int W,
                                                        int Eloc, const int32_t* __restrict__ send_map,
                                                        int32_t* __restrict__ send_ids) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (p >= tokens * W) return;
   const int32_t row = send_map[p];
@@ -207,13 +210,16 @@ extern "C" fp8q_status fp8q_ep_dispatch_pack(const uint8_t* xq, const uint8_t* x
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   fp8q_status rs = route_pairs(dev, tokens, didx, W, W, 1, true, send_offsets, send_map, route_ws, st);
   if (rs != FP8Q_OK) return rs;
-  if (hidden > 0) {
-    rs = launch_scatter_copy(xq, xsf, tokens, hidden, send_map, W, W, 1, send_q, send_sf, send_offsets,
-                             route_totals(route_ws, tokens, W, W), st);
-    if (rs != FP8Q_OK) return rs;
-  }
-  send_ids_kernel<<<(unsigned)((npairs + 255) / 256), 256, 0, st>>>(topk_idx, tokens, K, W, Eloc, send_map, send_ids);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  // The slot ids need only the send map; launched before the payload (both as dependent
+  // launches), so the payload's loads overlap them.
+  const int32_t* smap = send_map;
+  if (launch_after(send_ids_kernel, (unsigned)((npairs + 255) / 256), 256, 0, st, topk_idx, tokens, K, W, Eloc, smap,
+                   send_ids) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (hidden > 0)
+    return launch_scatter_copy(xq, xsf, tokens, hidden, send_map, W, W, 1, send_q, send_sf, send_offsets,
+                               route_totals(route_ws, tokens, W, W), st);
+  return FP8Q_OK;
 }
 
 extern "C" fp8q_status fp8q_ep_recv_permute_fp8(const fp8q_ep_source* sources, int32_t num_sources, int64_t hidden,

@@ -20,7 +20,8 @@
 // packed word before the kernel's one barrier; every thread then assembles the two words
 // of maxima it needs with byte permutes.  The shift of a 16-byte row chunk uses its own
 // 32x32 block's k; staging and the byte transpose (8 tokens x 8 channels per lane) are
-// those of the 128 kernel.
+// those of the 128 kernel.  A 2-D grid (column blocks x row blocks); the shift's form is chosen
+// once per warp (shift_row16_warp).
 #include "common.cuh"
 #include "launch.h"
 
@@ -84,8 +85,8 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const int ngr = cols >> 5;  // scale bytes per row
-  const int64_t b = (int64_t)blockIdx.x / ncb;
-  const int j = (int)((int64_t)blockIdx.x - b * ncb);
+  const int64_t b = blockIdx.y;  // 2-D grid: column blocks x row blocks
+  const int j = blockIdx.x;
   const int64_t r0 = b * 128;
   const int c0 = j * 128;
   const int sub = tid & 7, rsub = tid >> 3;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   for (int p = 0; p < kPasses; ++p) {
     const int rl = p * 32 + rsub;  // row group p
     uint32_t w[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
-    shift_row16(w, byte_of(smax_mine, p) - byte_of(e_row[rl], cg));
+    shift_row16_warp(w, byte_of(smax_mine, p) - byte_of(e_row[rl], cg));
     *reinterpret_cast<uint4*>(tile + rl * 128 + 16 * chunk_pos(rl, sub)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   __syncthreads();
@@ -165,7 +166,9 @@ fp8q_status launch_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, in
   const int64_t nblk = (rows / 128) * (cols / 128);
   if (nblk == 0) return FP8Q_OK;
   if (nblk > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  direct_transpose_mx32_kernel<<<(unsigned)nblk, kThreads, 0, stream>>>(q, sf, rows, (int)cols, qt, sft);
+  if (rows / 128 > 65535) return FP8Q_ERR_SHAPE;  // grid y limit (rows up to 8,388,480)
+  direct_transpose_mx32_kernel<<<dim3((unsigned)(cols / 128), (unsigned)(rows / 128)), kThreads, 0, stream>>>(
+      q, sf, rows, (int)cols, qt, sft);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

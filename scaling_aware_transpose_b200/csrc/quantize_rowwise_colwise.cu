@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       }
     }
     if (kColwise) {
-      shift_row16(w, emax - e[p]);
+      shift_row16_warp(w, emax - e[p]);
       uint8_t* row = tile + rl * 128 + 8 * (sub & 1);
       *reinterpret_cast<uint2*>(row + 16 * tile_chunk(rl, sub >> 1)) = make_uint2(w[0], w[1]);
       *reinterpret_cast<uint2*>(row + 16 * tile_chunk(rl, 4 + (sub >> 1))) = make_uint2(w[2], w[3]);

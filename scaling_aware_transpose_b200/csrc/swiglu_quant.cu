@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
         w[i][1] = v.y;
         w[i][2] = v.z;
         w[i][3] = v.w;
-        shift_row16(w[i], emax - (int)((ew >> (8 * i)) & 0xFFu));
+        shift_row16_warp(w[i], emax - (int)((ew >> (8 * i)) & 0xFFu));
       }
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
