@@ -3,15 +3,20 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the hot path over one batch of the dense-activation workload
-(X bf16 [8192, 7168], N(0,1) times a lognormal(0, 1.5) row factor, 7 outlier channels
-x100): fp8q_quantize_rowwise (X -> Q, SF) then fp8q_direct_transpose (Q, SF -> Q^T, SF^T).
-Each kernel is timed with CUDA events on the launching stream after an L2 flush (a
-256 MiB device write, outside the events), so both read their inputs from HBM.  The
-metric is algorithmic HBM bytes / kernel time (every input byte read once, every output
-byte written once), in GB/s.  With N ranks (torchrun, one GPU each) every rank runs its
-own batch (weak scaling, no collective on the data path); the value is all ranks' bytes
-over the slowest rank's time.  Rank 0 prints one JSON line.
+One step = one pass of the hot path over the dense-activation workload (X bf16
+[8192, 7168], N(0,1) times a lognormal(0, 1.5) row factor, 7 outlier channels x100):
+fp8q_quantize_rowwise (X -> Q, SF) and fp8q_direct_transpose (Q, SF -> Q^T, SF^T).
+The kernels stream over four rotating buffer sets (944 MB, more than seven times the
+L2): step k quantizes set k mod 4 and transposes set (k - 2) mod 4, whose codes were
+written two steps (590 MB of traffic) earlier, so both kernels read their inputs from
+HBM and each pays for the write-back of the lines it displaces, as in a long run; every
+batch still goes through both kernels.  The K timed steps are bracketed by one pair of
+CUDA events on the launching stream, with nothing between the launches; each kernel's
+own duration (for the roofline) comes from K back-to-back launches of that kernel over
+the same sets, again in one event pair.  The metric is algorithmic HBM bytes / time
+(every input byte read once, every output byte written once), in GB/s.  With N ranks (torchrun, one GPU each) every rank runs its own batches (weak
+scaling, no collective on the data path); the value is all ranks' bytes over the
+slowest rank's time.  Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (plain C, the parity reference) on the host cores
 on a bounded sample of the same workload; only rank 0 runs it.
@@ -42,6 +47,8 @@ BYTES_MX_QUANT = 3 * N_ELEM + N_ELEM // 32                      # 1x32 tiles
 BYTES_MX_DIRECT = 2 * (N_ELEM + N_ELEM // 32)                   # 32x32 blocks
 METRIC = "direct-transpose & quantize GB/s on 1 B200 (% of HBM peak); bit-exact vs oracle"
 FLUSH_BYTES = 256 << 20
+SETS = 4   # rotating buffer sets of the timed loop
+LAG = 2    # the transpose of step k reads the codes quantized in step k - LAG
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -60,8 +67,13 @@ def kernel_sources(kind: str):
     csrc = os.path.join(ROOT, "scaling_aware_transpose_b200", "csrc")
     main = {"quantize": "quantize_rowwise.cu", "direct": "direct_transpose.cu", "swiglu": "swiglu_quant.cu",
             "permute": "permute_pad_quant.cu", "rowwise_colwise": "quantize_rowwise_colwise.cu",
-            "unpermute": "unpermute_unpad.cu", "unpermute_fp8": "unpermute_unpad.cu", "mx32": "mx32.cu"}[kind]
-    return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")]
+            "unpermute": "unpermute_unpad.cu", "unpermute_fp8": "unpermute_unpad.cu", "mx32": "mx32.cu",
+            "mx32_quantize": "mx32.cu", "direct_grouped": "direct_transpose.cu", "naive": "naive_transpose.cu",
+            "permute_fp8": "permute_pad_quant.cu", "ep_pack": "ep_dispatch.cu", "ep_recv": "ep_dispatch.cu"}[kind]
+    extra = ["permute_common.cuh", "permute_pad_quant.cu"] if kind in ("ep_pack", "ep_recv") else []
+    if kind in ("permute", "permute_fp8"):
+        extra = ["permute_common.cuh"]
+    return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")] + [os.path.join(csrc, e) for e in extra]
 
 
 def source_digest(paths) -> str:
@@ -202,107 +214,185 @@ def time_on_stream(fn, reps, stream, before=None):
     return statistics.median(a.elapsed_time(b) * 1e-3 for a, b in pairs)
 
 
-def measure_workloads(reps, device, stream, flush, peak):
-    """The other hot-path rows on their own workloads, each kernel after an L2 flush:
-    fused SwiGLU+quantize(+transpose) on gate/up [32768, 2048]; fused permute+pad(128)+
-    quantize of X [16384, 7168] with top-8 of 32 Zipf(1.1) experts, then the grouped
-    direct transpose on its device offsets, and the combine-side unpermute+unpad of BF16
-    expert outputs (weighted) and of the FP8 rows (unit weights); quantize + direct
-    transpose on the range-stress X [65536, 7168]."""
+def time_steady(calls, n, stream):
+    """Mean device time (s) of n back-to-back launches cycling over `calls` (one callable
+    per buffer set), bracketed by one pair of CUDA events on `stream`; nothing runs
+    between the launches."""
+    import torch
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(2_000_000)  # the host queues the launches while the GPU waits
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n):
+        calls[i % len(calls)]()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1e-3 / n
+
+
+def sets_for(bytes_per_set: int, l2_bytes: int) -> int:
+    """Buffer sets a steady-state loop cycles over: together at least three times the L2,
+    and never fewer than two (so no launch reads what the previous one touched)."""
+    return max(2, -(-3 * l2_bytes // max(bytes_per_set, 1)))
+
+
+def measure_workloads(reps, device, stream, peak):
+    """The other hot-path rows on their own workloads, each kernel timed in steady state
+    (back-to-back launches over rotating buffer sets, see time_steady): fused
+    SwiGLU+quantize(+transpose) on gate/up [32768, 2048]; fused permute+pad(128)+quantize
+    of X [16384, 7168] with top-8 of 32 Zipf(1.1) experts, the FP8-input permute, the
+    grouped direct transpose on the permute's device offsets, and the combine-side
+    unpermute+unpad of BF16 expert outputs (weighted) and of the FP8 rows (unit weights);
+    the expert-parallel dispatch of the same tokens over 4 ranks (pack on one source
+    rank, receive permute on one destination rank from four source segments); quantize +
+    direct transpose on the range-stress X [65536, 7168]."""
     import torch
 
     import scaling_aware_transpose_b200 as sat
     from scaling_aware_transpose_b200 import synthetic
     sp = stream.cuda_stream
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    n = max(6, reps)
 
-    def entry(nbytes, t):
+    def entry(nbytes, t, sets):
         gbs = nbytes / t / 1e9
         return {"us": round(t * 1e6, 2), "bytes": int(nbytes), "GB/s": round(gbs, 1),
-                "frac_of_peak": round(gbs / peak, 4)}
+                "frac_of_peak": round(gbs / peak, 4), "sets": sets}
+
+    def copies(t, k):
+        return [t] + [t.clone() for _ in range(k - 1)]
 
     out = {}
     # SwiGLU
     d = synthetic.swiglu()
-    g = synthetic.to_torch_bf16(d["gate"]).to(device)
-    u = synthetic.to_torch_bf16(d["up"]).to(device)
-    R, C = g.shape
-    n = R * C
-    q = torch.empty((R, C), dtype=torch.uint8, device=device)
-    sf = torch.empty((R, C // 128), dtype=torch.uint8, device=device)
-    qt = torch.empty((C, R), dtype=torch.uint8, device=device)
-    sft = torch.empty((C, R // 128), dtype=torch.uint8, device=device)
-    t = time_on_stream(lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, qt, sft, sp), reps + 2, stream,
-                       lambda: flush.fill_(5))
-    t_row = time_on_stream(lambda: sat.fp8q_swiglu_quant(g, u, R, C, q, sf, None, None, sp), reps + 2, stream,
-                           lambda: flush.fill_(5))
-    out["swiglu_quant [32768x2048] (+transpose)"] = entry(4 * n + 2 * (n + n // 128), t)
-    out["swiglu_quant [32768x2048] (row-wise only)"] = entry(4 * n + n + n // 128, t_row)
-    del g, u, q, sf, qt, sft
-    # MoE: permute + pad + quantize, grouped direct transpose
+    g0 = synthetic.to_torch_bf16(d["gate"]).to(device)
+    u0 = synthetic.to_torch_bf16(d["up"]).to(device)
+    R, C = g0.shape
+    ne = R * C
+    b_sw = 4 * ne + 2 * (ne + ne // 128)
+    S = sets_for(b_sw, l2)
+    g, u = copies(g0, S), copies(u0, S)
+    q = [torch.empty((R, C), dtype=torch.uint8, device=device) for _ in range(S)]
+    sf = [torch.empty((R, C // 128), dtype=torch.uint8, device=device) for _ in range(S)]
+    qt = [torch.empty((C, R), dtype=torch.uint8, device=device) for _ in range(S)]
+    sft = [torch.empty((C, R // 128), dtype=torch.uint8, device=device) for _ in range(S)]
+    t = time_steady([lambda i=i: sat.fp8q_swiglu_quant(g[i], u[i], R, C, q[i], sf[i], qt[i], sft[i], sp)
+                     for i in range(S)], n, stream)
+    t_row = time_steady([lambda i=i: sat.fp8q_swiglu_quant(g[i], u[i], R, C, q[i], sf[i], None, None, sp)
+                         for i in range(S)], n, stream)
+    out["swiglu_quant [32768x2048] (+transpose)"] = entry(b_sw, t, S)
+    out["swiglu_quant [32768x2048] (row-wise only)"] = entry(4 * ne + ne + ne // 128, t_row, S)
+    del g, u, q, sf, qt, sft, g0, u0
+    torch.cuda.empty_cache()
+    # MoE: permute + pad + quantize, FP8-input permute, grouped direct transpose, combine
     d = synthetic.moe()
-    x = synthetic.to_torch_bf16(d["x"]).to(device)
+    x0 = synthetic.to_torch_bf16(d["x"]).to(device)
     idx = torch.from_numpy(d["topk_idx"]).to(device)
-    T, H = x.shape
+    T, H = x0.shape
     K, E, align = idx.shape[1], d["num_experts"], 128
     max_rows = sat.permute_max_rows(T, K, E, align)
-    q = torch.empty((max_rows, H), dtype=torch.uint8, device=device)
-    sf = torch.empty((max_rows, H // 128), dtype=torch.uint8, device=device)
+    ws = torch.empty(sat.fp8q_permute_workspace_bytes(T, K, E), dtype=torch.uint8, device=device)
     off = torch.empty(E + 1, dtype=torch.int32, device=device)
     rmap = torch.empty(T * K, dtype=torch.int32, device=device)
-    ws = torch.empty(sat.fp8q_permute_workspace_bytes(T, K, E), dtype=torch.uint8, device=device)
-    perm = lambda: sat.fp8q_permute_pad_quant(x, T, H, idx, K, E, align, q, sf, max_rows, off, rmap, ws,
-                                              ws.numel(), sp)
-    t_perm = time_on_stream(perm, reps + 2, stream, lambda: flush.fill_(6))
+    S = 2
+    xs = copies(x0, S)
+    q = [torch.empty((max_rows, H), dtype=torch.uint8, device=device) for _ in range(S)]
+    sf = [torch.empty((max_rows, H // 128), dtype=torch.uint8, device=device) for _ in range(S)]
+    t_perm = time_steady([lambda i=i: sat.fp8q_permute_pad_quant(xs[i], T, H, idx, K, E, align, q[i], sf[i], max_rows,
+                                                                 off, rmap, ws, ws.numel(), sp) for i in range(S)],
+                         n, stream)
     R = int(off[-1].item())
-    # FP8-input permute (the dispatch delivered row-wise codes and scales): same routing,
-    # rows copied instead of quantized
-    xq, xsf = sat.quantize_rowwise(x)
-    q8 = torch.empty_like(q)
-    sf8 = torch.empty_like(sf)
-    perm8 = lambda: sat.fp8q_permute_pad_fp8(xq, xsf, T, H, idx, K, E, align, q8, sf8, max_rows, off, rmap, ws,
-                                             ws.numel(), sp)
-    t_perm8 = time_on_stream(perm8, reps + 2, stream, lambda: flush.fill_(14))
-    del xq, xsf, q8, sf8
-    qt = torch.empty(max_rows * H, dtype=torch.uint8, device=device)
-    sft = torch.empty(max_rows * H // 128, dtype=torch.uint8, device=device)
-    t_gt = time_on_stream(lambda: sat.fp8q_direct_transpose(q, sf, max_rows, H, off, E, qt, sft, sp), reps + 2,
-                          stream, lambda: flush.fill_(7))
+    # FP8-input permute (the dispatch delivered row-wise codes and scales)
+    xq0, xsf0 = sat.quantize_rowwise(x0)
+    xq, xsf = copies(xq0, S), copies(xsf0, S)
+    q8 = [torch.empty_like(q[0]) for _ in range(S)]
+    sf8 = [torch.empty_like(sf[0]) for _ in range(S)]
+    t_perm8 = time_steady([lambda i=i: sat.fp8q_permute_pad_fp8(xq[i], xsf[i], T, H, idx, K, E, align, q8[i], sf8[i],
+                                                                max_rows, off, rmap, ws, ws.numel(), sp)
+                           for i in range(S)], n, stream)
+    del q8, sf8
+    torch.cuda.empty_cache()
+    qt = [torch.empty(max_rows * H, dtype=torch.uint8, device=device) for _ in range(S)]
+    sft = [torch.empty(max_rows * H // 128, dtype=torch.uint8, device=device) for _ in range(S)]
+    t_gt = time_steady([lambda i=i: sat.fp8q_direct_transpose(q[i], sf[i], max_rows, H, off, E, qt[i], sft[i], sp)
+                        for i in range(S)], n, stream)
     perm_bytes = 2 * T * H + 4 * T * K + R * (H + H // 128) + 4 * (E + 1) + 4 * T * K
-    out[f"permute_pad_quant [16384x7168] top8/32 -> {R} rows"] = entry(perm_bytes, t_perm)
+    out[f"permute_pad_quant [16384x7168] top8/32 -> {R} rows"] = entry(perm_bytes, t_perm, S)
     perm8_bytes = T * (H + H // 128) + 4 * T * K + R * (H + H // 128) + 4 * (E + 1) + 4 * T * K
-    out[f"permute_pad_fp8 [16384x7168] top8/32 -> {R} rows"] = entry(perm8_bytes, t_perm8)
-    out[f"direct_transpose grouped [{R}x7168] 32 experts"] = entry(2 * R * (H + H // 128), t_gt)
+    out[f"permute_pad_fp8 [16384x7168] top8/32 -> {R} rows"] = entry(perm8_bytes, t_perm8, S)
+    out[f"direct_transpose grouped [{R}x7168] 32 experts"] = entry(2 * R * (H + H // 128), t_gt, S)
     del qt, sft
+    torch.cuda.empty_cache()
     # combine side: unpermute + unpad of BF16 expert outputs with routing weights, and of
     # the FP8 rows with unit weights (the permute's backward shape)
     c = synthetic.moe_combine(rows=R, topk=K)
-    y = synthetic.to_torch_bf16(c["y"]).to(device)
+    y0 = synthetic.to_torch_bf16(c["y"]).to(device)
+    ys = copies(y0, S)
     wts = torch.from_numpy(c["weights"]).to(device)
-    comb = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-    t_ub = time_on_stream(lambda: sat.fp8q_unpermute_unpad(y, None, R, H, rmap, wts, T, K, comb, sp), reps + 2,
-                          stream, lambda: flush.fill_(12))
-    t_uq = time_on_stream(lambda: sat.fp8q_unpermute_unpad(q, sf, max_rows, H, rmap, None, T, K, comb, sp), reps + 2,
-                          stream, lambda: flush.fill_(13))
+    comb = [torch.empty((T, H), dtype=torch.bfloat16, device=device) for _ in range(S)]
+    t_ub = time_steady([lambda i=i: sat.fp8q_unpermute_unpad(ys[i], None, R, H, rmap, wts, T, K, comb[i], sp)
+                        for i in range(S)], n, stream)
+    t_uq = time_steady([lambda i=i: sat.fp8q_unpermute_unpad(q[i], sf[i], max_rows, H, rmap, None, T, K, comb[i], sp)
+                        for i in range(S)], n, stream)
     out[f"unpermute_unpad bf16 [{R}x7168] -> [16384x7168], weighted"] = entry(
-        T * K * 2 * H + 2 * T * H + 8 * T * K, t_ub)
+        T * K * 2 * H + 2 * T * H + 8 * T * K, t_ub, S)
     out[f"unpermute_unpad fp8 [{R}x7168] -> [16384x7168], unit weights"] = entry(
-        T * K * (H + H // 128) + 2 * T * H + 4 * T * K, t_uq)
-    del x, idx, q, sf, off, rmap, ws, y, wts, comb
+        T * K * (H + H // 128) + 2 * T * H + 4 * T * K, t_uq, S)
+    del ys, y0, comb, q, sf, xs
+    torch.cuda.empty_cache()
+    # expert-parallel dispatch of the same tokens over 4 ranks of 8 experts: the send-side
+    # pack of rank 0's 4096 tokens, and rank 0's receive permute from four source segments
+    # (the four ranks' send buffers, read in place as an all-to-all receive buffer would be)
+    W, Tr = 4, T // 4
+    Eloc = E // W
+    packs = [sat.ep_dispatch_pack(xq0[r * Tr:(r + 1) * Tr], xsf0[r * Tr:(r + 1) * Tr], idx[r * Tr:(r + 1) * Tr], W,
+                                  Eloc) for r in range(W)]
+    torch.cuda.synchronize()
+    offs = [p[3].tolist() for p in packs]
+    sent0 = offs[0][W]
+    pk_ws = torch.empty(sat.fp8q_ep_pack_workspace_bytes(Tr, W), dtype=torch.uint8, device=device)
+    pk_out = packs[0][:5]
+    xq_r, xsf_r, idx_r = xq0[:Tr], xsf0[:Tr], idx[:Tr]
+    t_pack = time_steady([lambda: sat.fp8q_ep_dispatch_pack(xq_r, xsf_r, Tr, H, idx_r, K, W, Eloc, pk_out[0], pk_out[1],
+                                                            pk_out[2], pk_out[0].shape[0], pk_out[3], pk_out[4], pk_ws,
+                                                            pk_ws.numel(), sp)], n, stream)
+    segs = [(p[0][o[0]:o[1]], p[1][o[0]:o[1]], p[2][o[0]:o[1]]) for p, o in zip(packs, offs)]
+    Rr = sum(sg[0].shape[0] for sg in segs)
+    rq, rsf, roff, rrmap = sat.ep_recv_permute(segs, Eloc, align)
+    rws = torch.empty(sat.fp8q_ep_recv_workspace_bytes(Rr, K, Eloc), dtype=torch.uint8, device=device)
+    seg_args = [(a, b_, c_, a.shape[0]) for a, b_, c_ in segs]
+    t_recv = time_steady([lambda: sat.fp8q_ep_recv_permute_fp8(seg_args, H, K, Eloc, align, rq, rsf, rq.shape[0], roff,
+                                                               rrmap, rws, rws.numel(), sp)], n, stream)
+    Rl = int(roff[-1].item())
+    local_slots = int((rrmap >= 0).sum().item())
+    out[f"ep_dispatch_pack rank 0 of 4: [{Tr}x7168] -> {sent0} rows"] = entry(
+        Tr * (H + H // 128) + 4 * Tr * K + sent0 * (H + H // 128 + 4 * K) + 4 * (W + 1) + 4 * Tr * W, t_pack, 1)
+    out[f"ep_recv_permute rank 0 of 4: {Rr} rows from 4 segments -> {Rl} rows"] = entry(
+        Rr * (H + H // 128 + 4 * K) + local_slots * (H + H // 128) + (Rl - local_slots) * (H + H // 128)
+        + 4 * (Eloc + 1) + 4 * Rr * K, t_recv, 1)
+    del packs, segs, seg_args, rq, rsf, xq, xsf, xq0, xsf0, x0
+    torch.cuda.empty_cache()
     # range stress
     d = synthetic.stress()
-    x = synthetic.to_torch_bf16(d["x"]).to(device)
-    R, C = x.shape
-    n = R * C
-    q = torch.empty((R, C), dtype=torch.uint8, device=device)
-    sf = torch.empty((R, C // 128), dtype=torch.uint8, device=device)
-    qt = torch.empty((C, R), dtype=torch.uint8, device=device)
-    sft = torch.empty((C, R // 128), dtype=torch.uint8, device=device)
-    t_q = time_on_stream(lambda: sat.fp8q_quantize_rowwise(x, R, C, q, sf, sp), reps + 2, stream,
-                         lambda: flush.fill_(8))
-    t_d = time_on_stream(lambda: sat.fp8q_direct_transpose(q, sf, R, C, None, 1, qt, sft, sp), reps + 2, stream,
-                         lambda: flush.fill_(9))
-    out["quantize_rowwise stress [65536x7168]"] = entry(3 * n + n // 128, t_q)
-    out["direct_transpose stress [65536x7168]"] = entry(2 * n + 2 * (n // 128), t_d)
+    x0 = synthetic.to_torch_bf16(d["x"]).to(device)
+    R, C = x0.shape
+    ne = R * C
+    S = 2
+    xs = copies(x0, S)
+    q = [torch.empty((R, C), dtype=torch.uint8, device=device) for _ in range(S)]
+    sf = [torch.empty((R, C // 128), dtype=torch.uint8, device=device) for _ in range(S)]
+    qt = [torch.empty((C, R), dtype=torch.uint8, device=device) for _ in range(S)]
+    sft = [torch.empty((C, R // 128), dtype=torch.uint8, device=device) for _ in range(S)]
+    t_q = time_steady([lambda i=i: sat.fp8q_quantize_rowwise(xs[i], R, C, q[i], sf[i], sp) for i in range(S)], n,
+                      stream)
+    t_d = time_steady([lambda i=i: sat.fp8q_direct_transpose(q[i], sf[i], R, C, None, 1, qt[i], sft[i], sp)
+                       for i in range(S)], n, stream)
+    out["quantize_rowwise stress [65536x7168]"] = entry(3 * ne + ne // 128, t_q, S)
+    out["direct_transpose stress [65536x7168]"] = entry(2 * ne + 2 * (ne // 128), t_d, S)
+    del xs, q, sf, qt, sft, x0
+    torch.cuda.empty_cache()
     status = sat.fp8q_last_device_status(sp)
     if status != 0:
         raise RuntimeError(f"device status {sat.STATUS.get(status)} in the workload measurements")
@@ -388,87 +478,107 @@ def run_ours(args, rank, world, local_rank):
     sat.lib()  # fail loudly here if the library is missing
     x_bits = synthetic.dense(seed=rank)["x"]
     x_host = synthetic.to_torch_bf16(x_bits).pin_memory()
-    x = x_host.to(device)
-    q = torch.empty((ROWS, COLS), dtype=torch.uint8, device=device)
-    sf = torch.empty((ROWS, COLS // 128), dtype=torch.uint8, device=device)
-    qt = torch.empty((COLS, ROWS), dtype=torch.uint8, device=device)
-    sft = torch.empty((COLS, ROWS // 128), dtype=torch.uint8, device=device)
+    xs = [x_host.to(device) for _ in range(SETS)]
+    qs = [torch.empty((ROWS, COLS), dtype=torch.uint8, device=device) for _ in range(SETS)]
+    sfs = [torch.empty((ROWS, COLS // 128), dtype=torch.uint8, device=device) for _ in range(SETS)]
+    qts = [torch.empty((COLS, ROWS), dtype=torch.uint8, device=device) for _ in range(SETS)]
+    sfts = [torch.empty((COLS, ROWS // 128), dtype=torch.uint8, device=device) for _ in range(SETS)]
+    x, q, sf, qt, sft = xs[0], qs[0], sfs[0], qts[0], sfts[0]
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     sp = stream.cuda_stream
 
-    def quant():
-        sat.fp8q_quantize_rowwise(x, ROWS, COLS, q, sf, sp)
+    def quant(i=0):
+        sat.fp8q_quantize_rowwise(xs[i], ROWS, COLS, qs[i], sfs[i], sp)
 
-    def direct():
-        sat.fp8q_direct_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, sp)
+    def direct(i=0):
+        sat.fp8q_direct_transpose(qs[i], sfs[i], ROWS, COLS, None, 1, qts[i], sfts[i], sp)
 
-    def step(evs=None):
-        flush.fill_(1)
+    def step(k, evs=None):
+        a, b = k % SETS, (k - LAG) % SETS
         if evs:
             evs[0].record(stream)
-        quant()
+        quant(a)
         if evs:
             evs[1].record(stream)
-        flush.fill_(2)
-        if evs:
             evs[2].record(stream)
-        direct()
+        direct(b)
         if evs:
             evs[3].record(stream)
 
+    for i in range(SETS):
+        quant(i)
     W = max(3, args.warmup)
-    for _ in range(W):
-        step()
+    for k in range(W):
+        step(k)
     torch.cuda.synchronize()
     if sat.fp8q_last_device_status(sp) != 0:
         raise RuntimeError("device status set during warm-up")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    torch.cuda._sleep(2_000_000)  # the host queues the first launches while the GPU waits
     with ClockSampler(local_rank) as clocks:
+        t_start.record(stream)
         for k in range(K):
-            step(evs[k])
+            step(W + k)
+        t_end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    tq = [e[0].elapsed_time(e[1]) * 1e-3 for e in evs]
-    td = [e[2].elapsed_time(e[3]) * 1e-3 for e in evs]
-    total = sum(tq) + sum(td)
+    total = t_start.elapsed_time(t_end) * 1e-3
     total_max = reduce_max(total, dist, device)
+    # per-kernel durations: each kernel alone, the same number of back-to-back launches
+    # over the same rotating sets in one event pair (an event between two kernels costs
+    # the second one its launch overlap, about 3 us, so none is placed there)
+    def steady(fn, n):
+        fn(0)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n):
+            fn(i % SETS)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e-3 / n
+    t_q_steady = reduce_max(steady(quant, K), dist, device)
+    t_d_steady = reduce_max(steady(direct, K), dist, device)
+    # the same two kernels with an event pair around each one (the previous convention)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(min(K, 50))]
+    torch.cuda._sleep(2_000_000)
+    for k, e in enumerate(evs):
+        step(k, e)
+    torch.cuda.synchronize()
+    t_q_ev = statistics.median(e[0].elapsed_time(e[1]) * 1e-3 for e in evs)
+    t_d_ev = statistics.median(e[2].elapsed_time(e[3]) * 1e-3 for e in evs)
     status = sat.fp8q_last_device_status(sp)
     if status != 0:
         raise RuntimeError(f"device status {sat.STATUS.get(status)} after the timed region")
 
-    # ---- extra, untimed-by-the-headline measurements
-    # back-to-back step (no flush between the two kernels: Q stays in L2)
-    chained = []
-    for _ in range(min(K, 50)):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        flush.fill_(3)
-        a.record(stream)
-        quant()
-        direct()
-        b.record(stream)
-        chained.append((a, b))
-    # naive three-pass path on the same Q, SF
-    ws = torch.empty(sat.fp8q_naive_workspace_bytes(ROWS, COLS), dtype=torch.uint8, device=device)
-    nqt, nsft = torch.empty_like(qt), torch.empty_like(sft)
-    naive = []
-    for i in range(min(K, 50) + 3):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        flush.fill_(4)
-        a.record(stream)
-        sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, nqt, nsft, ws, ws.numel(), sp)
-        b.record(stream)
-        if i >= 3:
-            naive.append((a, b))
+    # every set's outputs are the same bytes: check set 0 against the others
     torch.cuda.synchronize()
-    t_chain = statistics.median(a.elapsed_time(b) * 1e-3 for a, b in chained)
-    t_naive = statistics.median(a.elapsed_time(b) * 1e-3 for a, b in naive)
+    same_sets = all(torch.equal(qts[i], qt) and torch.equal(sfts[i], sft) and torch.equal(qs[i], q)
+                    for i in range(1, SETS))
+
+    # ---- extra, untimed-by-the-headline measurements
+    # the earlier convention: a 256 MiB device write before each kernel, outside the
+    # events (it leaves L2 full of dirty lines whose write-back the kernel then pays)
+    t_q_dirty = time_on_stream(quant, min(K, 50), stream, lambda: flush.fill_(1))
+    t_d_dirty = time_on_stream(direct, min(K, 50), stream, lambda: flush.fill_(2))
+    # chained step: the transpose right after the quantize of the same set (Q still in L2),
+    # back to back over the rotating sets
+    t_chain = steady(lambda i: (quant(i), direct(i)), min(K, 100))
+    # naive three-pass path, back to back over the same rotating sets (its workspace is
+    # shared; each call moves about 590 MB)
+    ws = torch.empty(sat.fp8q_naive_workspace_bytes(ROWS, COLS), dtype=torch.uint8, device=device)
+    t_naive = steady(lambda i: sat.fp8q_naive_transpose(qs[i], sfs[i], ROWS, COLS, None, 1, qts[i], sfts[i], ws,
+                                                        ws.numel(), sp), min(K, 50))
+    for i in range(SETS):  # restore the sets' outputs for the checks below
+        direct(i)
 
     # same two kernels after a flush that leaves no dirty lines (write, then read the
     # flush buffer): the kernel does not pay for writing back data it never touched
@@ -479,27 +589,31 @@ def run_ours(args, rank, world, local_rank):
     t_d_clean = time_on_stream(direct, min(K, 50), stream, clean_flush)
 
     # single-pass quantizer: the same four outputs from one read of X (byte-identical to
-    # the two-kernel step); also with packed UE8M0 scales and the zero-tile option
-    rc_q, rc_sf = torch.empty_like(q), torch.empty_like(sf)
-    rc_qt, rc_sft = torch.empty_like(qt), torch.empty_like(sft)
+    # the two-kernel step); also with packed UE8M0 scales and the zero-tile option.  Back
+    # to back over the rotating X sets, each with its own outputs.
+    rc_out = [(torch.empty_like(q), torch.empty_like(sf), torch.empty_like(qt), torch.empty_like(sft))
+              for _ in range(SETS)]
     pk_sf = torch.empty(sat.packed_sf_shape(ROWS, COLS), dtype=torch.int32, device=device)
     pk_sft = torch.empty(sat.packed_sf_shape(COLS, ROWS), dtype=torch.int32, device=device)
-    rowcol = lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, 0, rc_q, rc_sf, rc_qt, rc_sft, sp)
-    rowcol_pk = lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, sat.ZERO_TILE_MIN_SCALE |
-                                                          sat.SF_PACKED_UE8M0, rc_q, pk_sf, rc_qt, pk_sft, sp)
-    t_rc = time_on_stream(rowcol, min(K, 50) + 3, stream, lambda: flush.fill_(10))
-    t_rc_clean = time_on_stream(rowcol, min(K, 50) + 3, stream, clean_flush)
-    t_rc_pk = time_on_stream(rowcol_pk, min(K, 50) + 3, stream, lambda: flush.fill_(11))
-    # MX granularity: 1x32 tiles and 32x32 transpose blocks on the same X
-    mq, msf = torch.empty_like(q), torch.empty((ROWS, COLS // 32), dtype=torch.uint8, device=device)
-    mqt, msft = torch.empty_like(qt), torch.empty((COLS, ROWS // 32), dtype=torch.uint8, device=device)
-    t_mxq = time_on_stream(lambda: sat.fp8q_quantize_rowwise_mx32(x, ROWS, COLS, mq, msf, sp), min(K, 50) + 3, stream,
-                           lambda: flush.fill_(15))
-    t_mxd = time_on_stream(lambda: sat.fp8q_direct_transpose_mx32(mq, msf, ROWS, COLS, mqt, msft, sp),
-                           min(K, 50) + 3, stream, lambda: flush.fill_(16))
-    del mq, msf, mqt, msft
-    rowcol()
+    rowcol = lambda i: sat.fp8q_quantize_rowwise_colwise(xs[i], ROWS, COLS, 0, *rc_out[i], sp)
+    rowcol_pk = lambda i: sat.fp8q_quantize_rowwise_colwise(xs[i], ROWS, COLS, sat.ZERO_TILE_MIN_SCALE |
+                                                            sat.SF_PACKED_UE8M0, rc_out[i][0], pk_sf, rc_out[i][2],
+                                                            pk_sft, sp)
+    t_rc = steady(rowcol, min(K, 100))
+    t_rc_pk = steady(rowcol_pk, min(K, 100))
+    t_rc_dirty = time_on_stream(lambda: rowcol(0), min(K, 50) + 3, stream, lambda: flush.fill_(10))
+    # MX granularity: 1x32 tiles and 32x32 transpose blocks on the same X, back to back
+    # over the rotating sets
+    mx = [(torch.empty_like(q), torch.empty((ROWS, COLS // 32), dtype=torch.uint8, device=device),
+           torch.empty_like(qt), torch.empty((COLS, ROWS // 32), dtype=torch.uint8, device=device))
+          for _ in range(SETS)]
+    t_mxq = steady(lambda i: sat.fp8q_quantize_rowwise_mx32(xs[i], ROWS, COLS, mx[i][0], mx[i][1], sp), min(K, 100))
+    t_mxd = steady(lambda i: sat.fp8q_direct_transpose_mx32(mx[i][0], mx[i][1], ROWS, COLS, mx[i][2], mx[i][3], sp),
+                   min(K, 100))
+    del mx
+    rowcol(0)
     torch.cuda.synchronize()
+    rc_q, rc_sf, rc_qt, rc_sft = rc_out[0]
     same_rc = all(torch.equal(a_, b_) for a_, b_ in ((rc_q, q), (rc_sf, sf), (rc_qt, qt), (rc_sft, sft)))
 
     # ---- end to end through the C ABI from pinned host buffers
@@ -534,7 +648,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
     peak, peak_kind = measured_peak_gbs()
-    avg_q, avg_d = sum(tq) / K, sum(td) / K
+    avg_q, avg_d = t_q_steady, t_d_steady
     dominant = "quantize" if avg_q >= avg_d else "direct"
     rf = roofline(BYTES_QUANT if dominant == "quantize" else BYTES_DIRECT, max(avg_q, avg_d), peak, peak_kind,
                   profiled_traffic(dominant))
@@ -546,8 +660,10 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": round(total_max / K * 1e3, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "path": "fp8q_quantize_rowwise -> fp8q_direct_transpose",
-                   "bytes_per_step": BYTES_STEP, "l2": "flushed before each kernel (256 MiB device write, "
-                   "outside the events)", "seed": "rank", "parallelism": f"replicas x{world} (no collective)"},
+                   "bytes_per_step": BYTES_STEP,
+                   "l2": f"inputs larger than L2: {SETS} rotating buffer sets ({SETS * BYTES_STEP // 10**6} MB); "
+                         f"step k quantizes set k and transposes set k-{LAG}, no flush",
+                   "seed": "rank", "parallelism": f"replicas x{world} (no collective)"},
         "roofline": rf,
         "kernels": {
             "quantize_rowwise": {"us": round(avg_q * 1e6, 2), "GB/s": round(BYTES_QUANT / avg_q / 1e9, 1),
@@ -558,23 +674,35 @@ def run_ours(args, rank, world, local_rank):
                                  "frac_of_peak": round(BYTES_DIRECT / avg_d / 1e9 / peak, 4),
                                  "frac_of_8000": round(BYTES_DIRECT / avg_d / 1e9 / 8000, 4),
                                  "traffic": profiled_traffic("direct")},
+            "per_kernel_timing": f"{K} back-to-back launches of one kernel over the {SETS} rotating sets, "
+                                 "one event pair (quantize_rowwise, direct_transpose above)",
+            "step_sum_vs_loop": round((avg_q + avg_d) / (total / K), 4),
+            "event_pair_per_kernel": {"quantize_us": round(t_q_ev * 1e6, 2), "direct_us": round(t_d_ev * 1e6, 2),
+                                      "how": "the headline loop with an event pair around each kernel"},
+            "dirty_l2_flush": {"quantize_us": round(t_q_dirty * 1e6, 2),
+                               "quantize_GB/s": round(BYTES_QUANT / t_q_dirty / 1e9, 1),
+                               "direct_us": round(t_d_dirty * 1e6, 2),
+                               "direct_GB/s": round(BYTES_DIRECT / t_d_dirty / 1e9, 1)},
+            "rotating_sets_outputs_identical": same_sets,
             "naive_transpose_3pass": {"us": round(t_naive * 1e6, 2),
                                       "GB/s_of_direct_bytes": round(BYTES_DIRECT / t_naive / 1e9, 1),
                                       "direct_speedup": round(t_naive / avg_d, 2)},
-            "chained_step_no_flush_between": {"us": round(t_chain * 1e6, 2),
-                                              "GB/s": round(BYTES_STEP / t_chain / 1e9, 1)},
+            "chained_step": {"us": round(t_chain * 1e6, 2), "GB/s": round(BYTES_STEP / t_chain / 1e9, 1),
+                             "how": "quantize then transpose of the same set (Q read back from L2), back to back "
+                                    "over the rotating sets"},
             "quantize_rowwise_colwise_single_pass": {
                 "us": round(t_rc * 1e6, 2), "bytes": BYTES_ROWCOL, "GB/s": round(BYTES_ROWCOL / t_rc / 1e9, 1),
                 "frac_of_peak": round(BYTES_ROWCOL / t_rc / 1e9 / peak, 4),
                 "frac_of_8000": round(BYTES_ROWCOL / t_rc / 1e9 / 8000, 4),
-                "clean_l2_us": round(t_rc_clean * 1e6, 2),
-                "clean_l2_GB/s": round(BYTES_ROWCOL / t_rc_clean / 1e9, 1),
+                "dirty_l2_flush_us": round(t_rc_dirty * 1e6, 2),
                 "packed_ue8m0_zero_tile_us": round(t_rc_pk * 1e6, 2),
                 "vs_two_kernel_step": round((avg_q + avg_d) / t_rc, 3),
                 "outputs_equal_two_kernel_step": same_rc,
                 "traffic": profiled_traffic("rowwise_colwise")},
             "mx32": {"quantize_us": round(t_mxq * 1e6, 2), "quantize_GB/s": round(BYTES_MX_QUANT / t_mxq / 1e9, 1),
-                     "direct_us": round(t_mxd * 1e6, 2), "direct_GB/s": round(BYTES_MX_DIRECT / t_mxd / 1e9, 1)},
+                     "quantize_frac_of_peak": round(BYTES_MX_QUANT / t_mxq / 1e9 / peak, 4),
+                     "direct_us": round(t_mxd * 1e6, 2), "direct_GB/s": round(BYTES_MX_DIRECT / t_mxd / 1e9, 1),
+                     "direct_frac_of_peak": round(BYTES_MX_DIRECT / t_mxd / 1e9 / peak, 4)},
             "clean_l2_flush": {"quantize_us": round(t_q_clean * 1e6, 2),
                                "quantize_GB/s": round(BYTES_QUANT / t_q_clean / 1e9, 1),
                                "direct_us": round(t_d_clean * 1e6, 2),
@@ -588,7 +716,9 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(),
     }
     if not args.no_extras:
-        line["workloads"] = measure_workloads(min(K, 20), device, stream, flush, peak)
+        del flush
+        torch.cuda.empty_cache()
+        line["workloads"] = measure_workloads(min(K, 20), device, stream, peak)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x_bits, budget_s=args.cpu_budget)
     return line
@@ -645,11 +775,36 @@ def run_profile(args):
             "naive": lambda: sat.fp8q_naive_transpose(q, sf, ROWS, COLS, None, 1, qt, sft, ws, ws.numel()),
             "rowwise_colwise": lambda: sat.fp8q_quantize_rowwise_colwise(x, ROWS, COLS, 0, q, sf, qt, sft),
         }
-    elif args.profile == "mx32":
+    elif args.profile in ("mx32", "mx32_quantize"):
         x = synthetic.to_torch_bf16(synthetic.dense(seed=0)["x"]).cuda()
         mq, msf = sat.quantize_rowwise_mx32(x)
         mqt, msft = sat.direct_transpose_mx32(mq, msf)
-        calls = {"mx32": lambda: sat.fp8q_direct_transpose_mx32(mq, msf, ROWS, COLS, mqt, msft)}
+        calls = {"mx32": lambda: sat.fp8q_direct_transpose_mx32(mq, msf, ROWS, COLS, mqt, msft),
+                 "mx32_quantize": lambda: sat.fp8q_quantize_rowwise_mx32(x, ROWS, COLS, mq, msf)}
+    elif args.profile == "direct_grouped":
+        d = synthetic.moe()
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        pq, psf, off, _ = sat.permute_pad_quant(x, idx, d["num_experts"], 128)
+        del x
+        qt = torch.empty(pq.numel(), dtype=torch.uint8, device="cuda")
+        sft = torch.empty(psf.numel(), dtype=torch.uint8, device="cuda")
+        R, H = pq.shape
+        calls = {"direct_grouped": lambda: sat.fp8q_direct_transpose(pq, psf, R, H, off, d["num_experts"], qt, sft)}
+    elif args.profile in ("ep_pack", "ep_recv"):
+        d = synthetic.moe()
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        xq, xsf = sat.quantize_rowwise(x)
+        del x
+        W, Tr = 4, xq.shape[0] // 4
+        Eloc = d["num_experts"] // W
+        packs = [sat.ep_dispatch_pack(xq[r * Tr:(r + 1) * Tr], xsf[r * Tr:(r + 1) * Tr], idx[r * Tr:(r + 1) * Tr],
+                                      W, Eloc) for r in range(W)]
+        offs = [p[3].tolist() for p in packs]
+        segs = [(p[0][o[0]:o[1]], p[1][o[0]:o[1]], p[2][o[0]:o[1]]) for p, o in zip(packs, offs)]
+        calls = {"ep_pack": lambda: sat.ep_dispatch_pack(xq[:Tr], xsf[:Tr], idx[:Tr], W, Eloc),
+                 "ep_recv": lambda: sat.ep_recv_permute(segs, Eloc, 128)}
     elif args.profile == "permute_fp8":
         d = synthetic.moe()
         x = synthetic.to_torch_bf16(d["x"]).cuda()
@@ -702,7 +857,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
     ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise",
-                                          "unpermute", "unpermute_fp8", "mx32", "permute_fp8"],
+                                          "unpermute", "unpermute_fp8", "mx32", "permute_fp8", "mx32_quantize",
+                                          "direct_grouped", "ep_pack", "ep_recv"],
                     default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)
