@@ -69,6 +69,7 @@ def kernel_sources(kind: str):
             "permute": "permute_pad_quant.cu", "rowwise_colwise": "quantize_rowwise_colwise.cu",
             "unpermute": "unpermute_unpad.cu", "unpermute_fp8": "unpermute_unpad.cu", "mx32": "mx32.cu",
             "mx32_quantize": "mx32.cu", "direct_grouped": "direct_transpose.cu", "naive": "naive_transpose.cu",
+            "direct_stress": "direct_transpose.cu",
             "permute_fp8": "permute_pad_quant.cu", "ep_pack": "ep_dispatch.cu", "ep_recv": "ep_dispatch.cu"}[kind]
     extra = ["permute_common.cuh", "permute_pad_quant.cu"] if kind in ("ep_pack", "ep_recv") else []
     if kind in ("permute", "permute_fp8"):
@@ -781,6 +782,13 @@ def run_profile(args):
         mqt, msft = sat.direct_transpose_mx32(mq, msf)
         calls = {"mx32": lambda: sat.fp8q_direct_transpose_mx32(mq, msf, ROWS, COLS, mqt, msft),
                  "mx32_quantize": lambda: sat.fp8q_quantize_rowwise_mx32(x, ROWS, COLS, mq, msf)}
+    elif args.profile == "direct_stress":
+        xs_ = synthetic.to_torch_bf16(synthetic.stress(seed=0)["x"]).cuda()
+        q, sf = sat.quantize_rowwise(xs_)
+        del xs_
+        qt, sft = sat.direct_transpose(q, sf)
+        R, H = q.shape
+        calls = {"direct_stress": lambda: sat.fp8q_direct_transpose(q, sf, R, H, None, 1, qt, sft)}
     elif args.profile == "direct_grouped":
         d = synthetic.moe()
         x = synthetic.to_torch_bf16(d["x"]).cuda()
@@ -858,7 +866,7 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
     ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise",
                                           "unpermute", "unpermute_fp8", "mx32", "permute_fp8", "mx32_quantize",
-                                          "direct_grouped", "ep_pack", "ep_recv"],
+                                          "direct_grouped", "ep_pack", "ep_recv", "direct_stress"],
                     default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)

@@ -68,7 +68,16 @@ def test_dense_config_full():
 
 
 def test_stress_config_full():
+    """65536 x 7168: large enough that the dense transpose takes its 256x128-tile kernel."""
     check_against_oracle(synthetic.stress()["x"])
+
+
+def test_large_tile_path_wide_rows():
+    """A second shape on the 256x128-tile kernel (at least eight waves of tiles): 6912 x
+    28672, 224 column blocks, range-stress tiles; and 6784 rows (not a multiple of 256),
+    which stays on the 128x128 kernel."""
+    for rows in (6912, 6784):
+        check_against_oracle(synthetic.stress(rows=rows, cols=28672, seed=rows)["x"])
 
 
 def test_all_bf16_values_at_fixed_scales():
