@@ -20,6 +20,18 @@
 // the token's row indices and weights are all loaded first: a thread's 16-byte FP8 chunk
 // takes as long to arrive as the index it depends on, so this saves a round trip per four
 // slots.  BF16 rows keep the index loads inside each batch, which measured faster there.
+//
+// FP8 rows with top-k <= 8 and hidden % 1024 == 0 take a warp-specialised ring instead
+// (unpermute_fp8_ring): one CTA per SM walks its tokens (blockIdx.x, + gridDim.x, ...)
+// through three shared-memory stages.  A producer warp keeps the next token's row
+// indices and weights in flight while it fills a stage: the token's K rows of codes
+// arrive by bulk copies (7 KB each at hidden 7168), its scale bytes by 8-byte cp.async,
+// both tracked by the stage's mbarrier; the consumer warps dequantize and accumulate from
+// shared memory in the same slot order as above (identical bytes) and release the stage
+// through a second mbarrier.  Row loads no longer wait on the index loads, and three
+// tokens' rows are in flight per SM without holding registers.  Every wait is bounded:
+// a timeout records FP8Q_ERR_TIMEOUT, raises an abort flag that stops both sides, and
+// the producer waits (bounded again) for the copies it issued before the CTA exits.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -172,6 +184,180 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
   dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// ---- FP8 ring (see the header)
+constexpr int kRingStages = 3;
+constexpr int kRingConsumerWarps = 14;
+constexpr int kRingThreads = (kRingConsumerWarps + 1) * 32;
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// Global -> shared bulk copy of `bytes` (16-byte aligned, a multiple of 16), completion
+// counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Stage bytes: codes [kK][hidden] | scale bytes [kK][hidden/128] (padded to 16) | row ids
+// int32 [kK] (-1: skipped) | weights fp32 [kK], rounded up to 128.
+__host__ __device__ inline int ring_stage_bytes(int K, int hidden) {
+  return (K * hidden + ((K * (hidden >> 7) + 15) & ~15) + 8 * K + 127) & ~127;
+}
+
+template <int kK>
+__global__ void __launch_bounds__(kRingThreads, 1) unpermute_fp8_ring(const uint8_t* __restrict__ y,
+                                                                      const uint8_t* __restrict__ y_sf, int64_t rows,
+                                                                      int hidden,
+                                                                      const int32_t* __restrict__ row_id_map,
+                                                                      const float* __restrict__ weights,
+                                                                      int64_t tokens, uint16_t* __restrict__ out,
+                                                                      int* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // stage filled: 32 async arrivals + 1 expect-tx arrival
+  uint64_t* empty = full + kRingStages;                 // stage released: one arrival per consumer warp
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kRingStages);
+  uint8_t* base = smem + 128;
+  const int ntile = hidden >> 7;
+  const int stage_bytes = ring_stage_bytes(kK, hidden);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int st = 0; st < kRingStages; ++st) {
+      mbar_init(&full[st], 33);
+      mbar_init(&empty[st], kRingConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int64_t ntok = tokens > (int64_t)blockIdx.x ? (tokens - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto stage = [&](int st, uint8_t*& codes, uint8_t*& scales, int32_t*& rowsel, float*& wsel) {
+    codes = base + (size_t)st * stage_bytes;
+    scales = codes + (size_t)kK * hidden;
+    rowsel = reinterpret_cast<int32_t*>(scales + ((kK * ntile + 15) & ~15));
+    wsel = reinterpret_cast<float*>(rowsel + kK);
+  };
+  if (warp == kRingConsumerWarps) {
+    // ---- producer warp
+    int64_t issued = 0;
+    int32_t r_next = -1;
+    float w_next = 1.0f;
+    if (ntok > 0 && lane < kK) {
+      r_next = __ldg(row_id_map + (int64_t)blockIdx.x * kK + lane);
+      w_next = weights != nullptr ? __ldg(weights + (int64_t)blockIdx.x * kK + lane) : 1.0f;
+    }
+    for (int64_t i = 0; i < ntok; ++i) {
+      const int st = (int)(i % kRingStages);
+      int32_t r = r_next;
+      const float w = w_next;
+      if (i + 1 < ntok && lane < kK) {  // the next token's indices, in flight while this one is issued
+        const int64_t tn = blockIdx.x + (i + 1) * gridDim.x;
+        r_next = __ldg(row_id_map + tn * kK + lane);
+        w_next = weights != nullptr ? __ldg(weights + tn * kK + lane) : 1.0f;
+      }
+      if (i >= kRingStages &&
+          !mbar_wait_bounded(&empty[st], (uint32_t)(((i / kRingStages) - 1) & 1), kWaitTimeoutNs)) {
+        if (lane == 0) record_status(status, FP8Q_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      uint8_t *codes, *scales;
+      int32_t* rowsel;
+      float* wsel;
+      stage(st, codes, scales, rowsel, wsel);
+      if (lane < kK) {
+        if (r < 0 || r >= rows) {
+          record_status(status, FP8Q_ERR_DEVICE);  // the slot is skipped
+          r = -1;
+        }
+        rowsel[lane] = r;
+        wsel[lane] = w;
+      }
+      const unsigned valid = __ballot_sync(0xFFFFFFFFu, lane < kK && r >= 0);
+      // scale rows in 8-byte pieces (hidden % 1024 == 0), spread over the lanes; every lane
+      // runs the same trip count so that the shuffle sees the whole warp
+      const int per_row = ntile >> 3;
+      for (int idx0 = 0; idx0 < kK * per_row; idx0 += 32) {
+        const int idx = idx0 + lane;
+        const int k = min(idx / per_row, kK - 1), piece = idx - k * per_row;
+        const int32_t rk = __shfl_sync(0xFFFFFFFFu, r, k);
+        if (idx < kK * per_row && rk >= 0)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(scales + k * ntile + 8 * piece)),
+                       "l"(y_sf + (int64_t)rk * ntile + 8 * piece)
+                       : "memory");
+      }
+      // this lane's arrival fires when its cp.asyncs have landed
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[st])) : "memory");
+      __syncwarp();  // orders every lane's row-id and weight stores before lane 0's release
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)(__popc(valid) * hidden));
+      if (lane < kK && r >= 0)
+        bulk_g2s(codes + (size_t)lane * hidden, y + (int64_t)r * hidden, (uint32_t)hidden, &full[st]);
+      issued = i + 1;
+    }
+    // Every copy this warp issued lands before the CTA may exit: wait (bounded) for the last
+    // phase issued on each stage.  On the normal path the consumers have already waited on
+    // them and these return at once.
+    for (int st = 0; st < kRingStages; ++st) {
+      if (issued <= st) continue;
+      const int64_t last = (issued - 1 - st) / kRingStages;  // phase index of stage st's last fill
+      if (!mbar_wait_bounded(&full[st], (uint32_t)(last & 1), kWaitTimeoutNs) && lane == 0)
+        record_status(status, FP8Q_ERR_TIMEOUT);
+    }
+    return;
+  }
+  // ---- consumer warps: 16 channels per thread and pass
+  const int nch = hidden >> 4;
+  for (int64_t i = 0; i < ntok; ++i) {
+    const int st = (int)(i % kRingStages);
+    if (!mbar_wait_bounded(&full[st], (uint32_t)((i / kRingStages) & 1), kWaitTimeoutNs)) {
+      if (lane == 0) record_status(status, FP8Q_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return;
+    }
+    if (*abort_flag != 0) return;
+    const int64_t t = blockIdx.x + i * gridDim.x;
+    uint8_t *codes, *scales;
+    int32_t* rowsel;
+    float* wsel;
+    stage(st, codes, scales, rowsel, wsel);
+    for (int c = tid; c < nch; c += kRingConsumerWarps * 32) {
+      float acc[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) acc[q] = -0.0f;
+#pragma unroll
+      for (int k = 0; k < kK; ++k) {
+        if (rowsel[k] < 0) continue;
+        const uint4 d = *reinterpret_cast<const uint4*>(codes + (size_t)k * hidden + 16 * c);
+        const float sc = ue8m0_scale(scales[k * ntile + (c >> 3)]);
+        const float wk = wsel[k];
+        float v[16];
+        dequant4(d.x, sc, v);
+        dequant4(d.y, sc, v + 4);
+        dequant4(d.z, sc, v + 8);
+        dequant4(d.w, sc, v + 12);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) acc[q] = __fmaf_rn(wk, v[q], acc[q]);
+      }
+      uint32_t o[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+        o[q] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(out + t * hidden + 16 * c);
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+}
+
 struct UnpermuteArgs {
   const uint8_t* y;
   const uint8_t* y_sf;
@@ -191,6 +377,15 @@ void launch_k(const UnpermuteArgs& a, unsigned blocks, cudaStream_t stream) {
                                                                     a.weights, a.tokens, a.topk, a.out, a.status);
 }
 
+template <int kK>
+cudaError_t launch_ring(const UnpermuteArgs& a, int grid, int smem, cudaStream_t stream) {
+  const cudaError_t e = cudaFuncSetAttribute(unpermute_fp8_ring<kK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  unpermute_fp8_ring<kK><<<grid, kRingThreads, smem, stream>>>(a.y, a.y_sf, a.rows, a.hidden, a.row_id_map, a.weights,
+                                                               a.tokens, a.out, a.status);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const uint8_t* y_sf, int64_t rows,
@@ -203,6 +398,23 @@ fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const u
   const unsigned blocks = (unsigned)blocks64;
   const UnpermuteArgs a{static_cast<const uint8_t*>(y), y_sf, rows, (int)hidden, row_id_map, weights, tokens, topk,
                         static_cast<uint16_t*>(out), dev.status};
+  const int ring_smem = 128 + kRingStages * ring_stage_bytes(topk, (int)hidden);
+  if (y_sf != nullptr && topk >= 1 && topk <= 8 && hidden % 1024 == 0 && ring_smem <= dev.max_smem_optin &&
+      (reinterpret_cast<uintptr_t>(y_sf) & 7u) == 0 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0) {
+    const int grid = (int)(tokens < dev.num_sms ? tokens : dev.num_sms);
+    cudaError_t e = cudaSuccess;
+    switch (topk) {
+      case 1: e = launch_ring<1>(a, grid, ring_smem, stream); break;
+      case 2: e = launch_ring<2>(a, grid, ring_smem, stream); break;
+      case 3: e = launch_ring<3>(a, grid, ring_smem, stream); break;
+      case 4: e = launch_ring<4>(a, grid, ring_smem, stream); break;
+      case 5: e = launch_ring<5>(a, grid, ring_smem, stream); break;
+      case 6: e = launch_ring<6>(a, grid, ring_smem, stream); break;
+      case 7: e = launch_ring<7>(a, grid, ring_smem, stream); break;
+      default: e = launch_ring<8>(a, grid, ring_smem, stream); break;
+    }
+    return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  }
   if (y_sf == nullptr) {
     launch_k<false, 0>(a, blocks, stream);
   } else {

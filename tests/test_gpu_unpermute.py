@@ -1,7 +1,8 @@
 """GPU parity of the fused unpermute + unpad (combine side of the permute) against the
 CPU oracle, byte for byte: BF16 and FP8 expert rows, routing weights and unit weights,
-K = 1..8 (each its own FP8 specialisation) and 12, 16, ragged hidden sizes, the permute round trip, the full MoE workload, and bad
-row indices reported through the status word."""
+K = 1..8 (each its own FP8 specialisation) and 12, 16, ragged hidden sizes, the FP8 bulk-copy ring
+(hidden % 1024 == 0, K <= 8), the permute round trip, the full MoE workload, and bad row indices reported
+through the status word."""
 import numpy as np
 import pytest
 import torch
@@ -34,6 +35,21 @@ def test_matches_oracle(fp8, weighted, T, H, K):
     y, sf, rmap, w = case(T, H, K, R, seed=T + H + K, fp8=fp8)
     w = w if weighted else None
     out = sat.unpermute_unpad(dev(y), dev(rmap), K, None if w is None else dev(w), None if sf is None else dev(sf))
+    device_status_ok()
+    assert_bytes_equal(host(out), oracle.unpermute_unpad(y, rmap, K, w, y_sf=sf), f"out T={T} H={H} K={K}")
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+@pytest.mark.parametrize("T,H,K", [(300, 1024, 1), (149, 1024, 2), (1000, 2048, 3), (5, 1024, 5), (777, 3072, 7),
+                                   (2000, 8192, 8), (160, 7168, 4), (148, 1024, 6)])
+def test_fp8_ring_matches_oracle(weighted, T, H, K):
+    """FP8 rows with top-k <= 8 and hidden % 1024 == 0 take the bulk-copy ring: fewer
+    tokens than SMs, exactly one per SM, and many tokens per CTA (the three stages wrap
+    around many times), every k, hidden up to 8192."""
+    R = T * K + 50
+    y, sf, rmap, w = case(T, H, K, R, seed=3 * T + H + K, fp8=True)
+    w = w if weighted else None
+    out = sat.unpermute_unpad(dev(y), dev(rmap), K, None if w is None else dev(w), dev(sf))
     device_status_ok()
     assert_bytes_equal(host(out), oracle.unpermute_unpad(y, rmap, K, w, y_sf=sf), f"out T={T} H={H} K={K}")
 
@@ -83,6 +99,15 @@ def test_bad_row_index_sets_device_status_fp8():
     q = torch.zeros((64, 256), dtype=torch.uint8, device="cuda")
     sf = torch.full((64, 2), 127, dtype=torch.uint8, device="cuda")
     for K, bad in ((2, [0, 1, 64, 3]), (8, list(range(15)) + [-1]), (12, list(range(23)) + [99])):
+        rmap = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        sat.unpermute_unpad(q, rmap, K, None, sf)
+        assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE, K
+    assert sat.fp8q_last_device_status() == 0
+    # the bulk-copy ring (hidden % 1024 == 0): a bad slot is skipped and reported, the rest
+    # of the token still combines
+    q = torch.zeros((64, 1024), dtype=torch.uint8, device="cuda")
+    sf = torch.full((64, 8), 127, dtype=torch.uint8, device="cuda")
+    for K, bad in ((2, [0, 1, 64, 3]), (8, list(range(15)) + [-1])):
         rmap = torch.tensor(bad, dtype=torch.int32, device="cuda")
         sat.unpermute_unpad(q, rmap, K, None, sf)
         assert sat.fp8q_last_device_status() == sat.FP8Q_ERR_DEVICE, K
