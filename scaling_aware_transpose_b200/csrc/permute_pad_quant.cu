@@ -233,6 +233,115 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
   }
 }
 
+// Rank with the scan folded in, for small routings (see route_pairs): the same stable
+// ranking as rank_multi_kernel, but each CTA derives its own bases from the per-chunk
+// histograms instead of reading them from scan_kernel.  A warp per group sums the group's
+// counts over all chunks (its total) and over the chunks before this one (this chunk's
+// prefix), lanes striding over the chunks; an exclusive scan of the padded totals over the
+// groups gives the offsets.  CTA 0 also writes offsets[0..E] and the totals, which the
+// payload's padding CTAs read.  The chain becomes histogram -> rank -> payload.
+__global__ void __launch_bounds__(kRankWarps * 32) rank_fused_kernel(const int32_t* __restrict__ idx, int64_t npairs,
+                                                                     int E, int align, const int32_t* __restrict__ counts,
+                                                                     int64_t C, int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ totals,
+                                                                     int32_t* __restrict__ row_id_map) {
+  extern __shared__ int32_t s_cnt[];  // [kRankWarps][E] | pre[E] | tot[E] | off[E] | warp sums[kRankWarps]
+  int32_t* s_pre = s_cnt + kRankWarps * E;
+  int32_t* s_tot = s_pre + E;
+  int32_t* s_off = s_tot + E;
+  int32_t* s_wsum = s_off + E;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  constexpr int kPer = kChunk / kRankWarps / 32;
+  const int64_t p0 = (int64_t)blockIdx.x * kChunk + w * (kChunk / kRankWarps);
+  int32_t ids[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    ids[i] = p < npairs ? __ldg(idx + p) : -1;
+  }
+  pdl_trigger();
+  for (int e = tid; e < kRankWarps * E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  int32_t* mine = s_cnt + w * E;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    const int32_t e = ids[i];
+    const bool ok = p < npairs && e >= 0 && e < E;
+    const unsigned same = __match_any_sync(0xFFFFFFFFu, ok ? e : -1 - lane);
+    if (ok && lane == __ffs(same) - 1) mine[e] += __popc(same);
+    __syncwarp();
+  }
+  pdl_wait();  // the histograms
+  for (int e = w; e < E; e += kRankWarps) {
+    int32_t tot = 0, pre = 0;
+    for (int64_t c = lane; c < C; c += 32) {
+      const int32_t v = __ldg(counts + c * E + e);
+      tot += v;
+      pre += c < (int64_t)blockIdx.x ? v : 0;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
+      pre += __shfl_xor_sync(0xFFFFFFFFu, pre, o);
+    }
+    if (lane == 0) {
+      s_tot[e] = tot;
+      s_pre[e] = pre;
+    }
+  }
+  __syncthreads();
+  // exclusive scan of the padded totals over the groups (E <= 512: two per thread)
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int32_t local = 0;
+  for (int e = e0; e < e1; ++e) local += (s_tot[e] + align - 1) / align * align;
+  const int32_t incl = warp_incl_scan32(local, lane);
+  if (lane == 31) s_wsum[w] = incl;
+  __syncthreads();
+  int32_t wbase = 0;
+  for (int ww = 0; ww < w; ++ww) wbase += s_wsum[ww];
+  int32_t run = wbase + incl - local;
+  for (int e = e0; e < e1; ++e) {
+    s_off[e] = run;
+    if (blockIdx.x == 0) {
+      offsets[e] = run;
+      totals[e] = s_tot[e];
+    }
+    run += (s_tot[e] + align - 1) / align * align;
+  }
+  if (blockIdx.x == 0 && tid == (int)blockDim.x - 1) offsets[E] = run;  // the last thread holds the total
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int32_t r = s_off[e] + s_pre[e];
+#pragma unroll
+    for (int ww = 0; ww < kRankWarps; ++ww) {
+      const int32_t v = s_cnt[ww * E + e];
+      s_cnt[ww * E + e] = r;
+      r += v;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t p = p0 + i * 32 + lane;
+    const bool live = p < npairs;
+    const int32_t e = ids[i];
+    const bool ok = live && e >= 0 && e < E;
+    const unsigned same = __match_any_sync(0xFFFFFFFFu, ok ? e : -1 - lane);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    const int base = ok ? mine[e] : 0;
+    __syncwarp();
+    if (ok) {
+      row_id_map[p] = base + rank;
+      if (lane == __ffs(same) - 1) mine[e] = base + __popc(same);
+    } else if (live) {
+      row_id_map[p] = -1;
+    }
+    __syncwarp();
+  }
+}
+
 // Tiles of x (token t, column block j) in row-major order: 8 lanes per tile, 16 bf16 per
 // lane (8 from each half of the tile), four tiles per warp per slot.  Each tile is read
 // and quantized once and its codes written to the token's top-k destination rows.
@@ -361,6 +470,15 @@ fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx,
   const size_t hist_smem = (size_t)E * sizeof(int32_t);
   count_kernel<<<(unsigned)C, 256, hist_smem, stream>>>(idx, npairs, E, allow_drop, counts, dev.status);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  // Small routings (at most 32 count loads per lane in the fused kernel's reduction) fold
+  // the one-CTA scan into the rank kernel: one dependent launch fewer.
+  if (E <= kRankMultiMaxE && (int64_t)((E + kRankWarps - 1) / kRankWarps) * ((C + 31) / 32) <= 32) {
+    const size_t smem = ((size_t)(kRankWarps + 3) * E + kRankWarps) * sizeof(int32_t);
+    return launch_after(rank_fused_kernel, (unsigned)C, kRankWarps * 32, smem, stream, idx, npairs, E, (int)align,
+                        (const int32_t*)counts, C, offsets, totals, row_id_map) == cudaSuccess
+               ? FP8Q_OK
+               : FP8Q_ERR_CUDA;
+  }
   if (launch_after(scan_kernel, 1, 1024, 0, stream, (const int32_t*)counts, C, E, (int)align, offsets, bases,
                    totals) != cudaSuccess)
     return FP8Q_ERR_CUDA;

@@ -97,6 +97,44 @@ def test_ep_many_ranks_and_empty_segments():
     run_ep(64, 20, 128, 2, 1, 16, seed=3)
 
 
+def test_ep_duplicate_experts_and_one_hot_rank():
+    """Routing the Zipf sampler never draws: two slots of a token on the same expert (one
+    send row, two slot ids, two expert rows), and every token routed to rank 2's experts
+    only (ranks 0, 1, 3 receive nothing)."""
+    W, T, H, K, Eloc, align = 4, 300, 256, 3, 4, 16
+    rng = np.random.default_rng(12)
+    xs = [oracle.quantize_rowwise(synthetic.scaled_normal(T, H, seed=40 + s)) for s in range(W)]
+    for mode in ("dup", "one_rank"):
+        idx = []
+        for s in range(W):
+            if mode == "dup":
+                a = rng.integers(0, W * Eloc, (T, K)).astype(np.int32)
+                a[:, 1] = a[:, 0]
+            else:
+                a = (2 * Eloc + rng.integers(0, Eloc, (T, K))).astype(np.int32)
+            idx.append(np.ascontiguousarray(a))
+        packs_d = [sat.ep_dispatch_pack(dev(xs[s][0]), dev(xs[s][1]), dev(idx[s]), W, Eloc) for s in range(W)]
+        device_status_ok()
+        packs_o = [oracle.ep_dispatch_pack(xs[s][0], xs[s][1], idx[s], W, Eloc) for s in range(W)]
+        for s in range(W):
+            _check_pack(packs_d[s], packs_o[s], T)
+        for d in range(W):
+            segs = [(p[0][int(o[3][d]):int(o[3][d + 1])], p[1][int(o[3][d]):int(o[3][d + 1])],
+                     p[2][int(o[3][d]):int(o[3][d + 1])]) for p, o in zip(packs_d, packs_o)]
+            q, sf, off, rmap = sat.ep_recv_permute(segs, Eloc, align)
+            device_status_ok()
+            rq = np.concatenate([p[0][p[3][d]:p[3][d + 1]] for p in packs_o])
+            rsf = np.concatenate([p[1][p[3][d]:p[3][d + 1]] for p in packs_o])
+            rids = np.concatenate([p[2][p[3][d]:p[3][d + 1]] for p in packs_o])
+            oq, osf, ooff, ormap = oracle.ep_recv_permute(rq, rsf, rids, Eloc, align)
+            assert_bytes_equal(host(off), ooff, f"{mode} rank {d} offsets")
+            n = int(ooff[-1])
+            if rq.shape[0]:
+                assert_bytes_equal(host(rmap), ormap, f"{mode} rank {d} row_id_map")
+            assert_bytes_equal(host(q)[:n], oq[:n], f"{mode} rank {d} Q")
+            assert_bytes_equal(host(sf)[:n], osf[:n], f"{mode} rank {d} SF")
+
+
 def test_ep_bad_ids_set_device_status():
     q = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
     sf = torch.full((4, 1), 127, dtype=torch.uint8, device="cuda")
