@@ -23,10 +23,14 @@
  *   - E4M3 codes are bytes (OCP E4M3FN: bias 7, max 448, no Inf).  Scales are UE8M0
  *     bytes: S = 2^(byte - 127).  An all-zero tile has scale byte 127 (S = 1).
  *   - Each call is asynchronous on `stream` (NULL = the legacy default stream) and
- *     returns after the launch.  Host-detectable argument errors return before any
- *     launch and leave every output untouched.  Errors that only the device can see
- *     (bad group offsets, routing indices out of range, a bounded wait that expired)
- *     are recorded in one per-device status word; read it with
+ *     returns after the launch.  Its kernels are launched as programmatic dependent
+ *     launches: their thread blocks may be placed on the GPU while the previous kernel
+ *     in the stream is finishing, but none touches memory before that kernel has
+ *     completed, so stream order holds as for a plain launch; a later kernel launched
+ *     the same way may likewise be placed early.  Host-detectable argument errors
+ *     return before any launch and leave every output untouched.  Errors that only the
+ *     device can see (bad group offsets, routing indices out of range, a bounded wait
+ *     that expired) are recorded in one per-device status word; read it with
  *     fp8q_last_device_status().
  *   - Inputs must be finite (no NaN/Inf); codes given to the transposes must come from
  *     a quantization (never 0x7F/0xFF).

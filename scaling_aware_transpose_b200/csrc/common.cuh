@@ -17,6 +17,36 @@ constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // bounded mbarrier waits: 1
 // First error wins; later ones are dropped so the reported code is the root cause.
 __device__ __forceinline__ void record_status(int* status, int code) { atomicCAS(status, 0, code); }
 
+// ------------------------------------------------------------ dependent launches
+// Every kernel of the library is launched with the programmatic-stream-serialization
+// attribute (launch_after), so its CTAs may be scheduled while the previous kernel in the
+// stream is still finishing.  pdl_wait() returns once that previous grid has completed
+// and its writes are visible (a hardware dependency, not a spin loop); pdl_trigger() lets
+// the next kernel in the stream be scheduled.  A kernel that begins a call waits before
+// its first global access and triggers after that wait, so whatever a later kernel of the
+// call reads before its own wait was complete before the call began.  Inside a call's
+// chain (routing -> payload) a kernel may trigger early and wait only where it first
+// reads its predecessor's output.  In a launch without the attribute, or after a kernel
+// that never triggers, both are no-ops and the launch is ordered as usual.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, unsigned block, size_t smem, cudaStream_t stream,
+                         Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------------ conversions
 // Two fp32 -> two E4M3 codes, round to nearest even, saturating to +-448; `lo` lands
 // in the low byte.

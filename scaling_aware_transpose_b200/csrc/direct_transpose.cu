@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kThreads, kGrouped ? 6 : 8) direct_transpose_k
                                                                      uint8_t* __restrict__ sft, int* status) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   int64_t b;
@@ -148,6 +150,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks2x1) direct_transpose_2x1(
   __shared__ __align__(128) uint8_t tile[256 * 128];
   __shared__ __align__(16) uint8_t e_row[256];
   __shared__ int emax_w[8];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const unsigned bq = blockIdx.x / (unsigned)ncb;
@@ -222,19 +226,23 @@ fp8q_status launch_direct_transpose(const DeviceInfo& dev, const uint8_t* q, con
   const int64_t nrb = rows / 128;
   const int64_t tiles2 = (rows / 256) * (cols / 128);
   if (!offsets && rows % 256 == 0 && tiles2 >= 8LL * kMinBlocks2x1 * dev.num_sms) {
-    direct_transpose_2x1<<<(unsigned)tiles2, kThreads, 0, stream>>>(q, sf, rows, (int)cols, qt, sft);
-    return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    return launch_after(direct_transpose_2x1, dim3((unsigned)tiles2), kThreads, 0, stream, q, sf, rows, (int)cols,
+                        qt, sft) == cudaSuccess
+               ? FP8Q_OK
+               : FP8Q_ERR_CUDA;
   }
+  const int32_t* no_offsets = nullptr;
+  cudaError_t rc;
   if (offsets)
-    direct_transpose_kernel<true><<<(unsigned)nblk, kThreads, 0, stream>>>(q, sf, rows, (int)cols, offsets, num_groups,
-                                                                           qt, sft, dev.status);
+    rc = launch_after(direct_transpose_kernel<true>, dim3((unsigned)nblk), kThreads, 0, stream, q, sf, rows, (int)cols,
+                      offsets, (int)num_groups, qt, sft, dev.status);
   else if (nrb > 1 && nrb <= 65535)  // 2-D grid: column blocks x row blocks
-    direct_transpose_kernel<false><<<dim3((unsigned)(cols / 128), (unsigned)nrb), kThreads, 0, stream>>>(
-        q, sf, rows, (int)cols, nullptr, 1, qt, sft, dev.status);
+    rc = launch_after(direct_transpose_kernel<false>, dim3((unsigned)(cols / 128), (unsigned)nrb), kThreads, 0, stream,
+                      q, sf, rows, (int)cols, no_offsets, 1, qt, sft, dev.status);
   else  // 1-D grid (gridDim.y == 1 selects the row-major mapping in the kernel)
-    direct_transpose_kernel<false><<<(unsigned)nblk, kThreads, 0, stream>>>(q, sf, rows, (int)cols, nullptr, 1, qt,
-                                                                            sft, dev.status);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    rc = launch_after(direct_transpose_kernel<false>, dim3((unsigned)nblk), kThreads, 0, stream, q, sf, rows, (int)cols,
+                      no_offsets, 1, qt, sft, dev.status);
+  return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 }  // namespace fp8q

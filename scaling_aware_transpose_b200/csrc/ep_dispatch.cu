@@ -54,6 +54,8 @@ __device__ __forceinline__ int segment_of(const int64_t* start, int n, int64_t x
 // d, else -1.  The d == 0 thread of each token checks the ids.
 __global__ void __launch_bounds__(256) dest_kernel(const int32_t* __restrict__ idx, int64_t tokens, int K, int W,
                                                    int Eloc, int32_t* __restrict__ didx, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (p >= tokens * W) return;
   const int64_t t = p / W;
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(256) send_ids_kernel(const int32_t* __restrict
 // Received slot ids of all segments -> one array [R * K] (the routing's input).
 __global__ void __launch_bounds__(256) gather_ids_kernel(const __grid_constant__ SegmentTable tab, int K,
                                                          int64_t npairs, int32_t* __restrict__ rid) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (p >= npairs) return;
   const int64_t r = p / K;
@@ -206,8 +210,9 @@ extern "C" fp8q_status fp8q_ep_dispatch_pack(const uint8_t* xq, const uint8_t* x
   int32_t* didx = static_cast<int32_t*>(workspace);
   void* route_ws = static_cast<uint8_t*>(workspace) + round16((size_t)(tokens * W) * sizeof(int32_t));
   const int64_t npairs = tokens * W;
-  dest_kernel<<<(unsigned)((npairs + 255) / 256), 256, 0, st>>>(topk_idx, tokens, K, W, Eloc, didx, dev.status);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (launch_after(dest_kernel, dim3((unsigned)((npairs + 255) / 256)), 256, 0, st, topk_idx, tokens, (int)K, (int)W,
+                   (int)Eloc, didx, dev.status) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
   fp8q_status rs = route_pairs(dev, tokens, didx, W, W, 1, true, send_offsets, send_map, route_ws, st);
   if (rs != FP8Q_OK) return rs;
   // The slot ids need only the send map; launched before the payload (both as dependent
@@ -279,8 +284,9 @@ extern "C" fp8q_status fp8q_ep_recv_permute_fp8(const fp8q_ep_source* sources, i
   int32_t* rid = static_cast<int32_t*>(workspace);
   void* route_ws = static_cast<uint8_t*>(workspace) + round16((size_t)(R * K) * sizeof(int32_t));
   const int64_t npairs = R * K;
-  gather_ids_kernel<<<(unsigned)((npairs + 255) / 256), 256, 0, st>>>(tab, K, npairs, rid);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (launch_after(gather_ids_kernel, dim3((unsigned)((npairs + 255) / 256)), 256, 0, st, tab, (int)K, npairs, rid) !=
+      cudaSuccess)
+    return FP8Q_ERR_CUDA;
   fp8q_status rs = route_pairs(dev, R, rid, K, Eloc, align, true, expert_offsets, row_id_map, route_ws, st);
   if (rs != FP8Q_OK || hidden == 0) return rs;
   const int pad_slots = (align - 1 + kPadRowsPerCta - 1) / kPadRowsPerCta;

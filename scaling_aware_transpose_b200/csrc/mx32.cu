@@ -39,6 +39,8 @@ __device__ __forceinline__ uint32_t chunk_maxabs(const uint4& v) {
 
 __global__ void __launch_bounds__(kQThreads) quantize_mx32_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
                                                                    uint8_t* __restrict__ sf, int64_t n_tiles) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * kQThreads + threadIdx.x) >> 5;
   uint4 v[kQUnroll][2];
@@ -82,6 +84,8 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ uint32_t e_row[128];  // 4 scale bytes of the row: column groups 0..3 of this tile
   __shared__ __align__(16) uint32_t smax_rg[4];  // row group rg: Smax byte of column groups 0..3
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const int ngr = cols >> 5;  // scale bytes per row
@@ -156,9 +160,10 @@ fp8q_status launch_quantize_mx32(const void* x, int64_t rows, int64_t cols, uint
   const int64_t tiles_per_block = (kQThreads / 32) * kQUnroll * 16;
   const int64_t blocks = (n_tiles + tiles_per_block - 1) / tiles_per_block;
   if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  quantize_mx32_kernel<<<(unsigned)blocks, kQThreads, 0, stream>>>(static_cast<const uint4*>(x),
-                                                                   reinterpret_cast<uint2*>(q), sf, n_tiles);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  return launch_after(quantize_mx32_kernel, dim3((unsigned)blocks), kQThreads, 0, stream,
+                      static_cast<const uint4*>(x), reinterpret_cast<uint2*>(q), sf, n_tiles) == cudaSuccess
+             ? FP8Q_OK
+             : FP8Q_ERR_CUDA;
 }
 
 fp8q_status launch_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t cols, uint8_t* qt,
@@ -167,9 +172,10 @@ fp8q_status launch_direct_transpose_mx32(const uint8_t* q, const uint8_t* sf, in
   if (nblk == 0) return FP8Q_OK;
   if (nblk > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   if (rows / 128 > 65535) return FP8Q_ERR_SHAPE;  // grid y limit (rows up to 8,388,480)
-  direct_transpose_mx32_kernel<<<dim3((unsigned)(cols / 128), (unsigned)(rows / 128)), kThreads, 0, stream>>>(
-      q, sf, rows, (int)cols, qt, sft);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  return launch_after(direct_transpose_mx32_kernel, dim3((unsigned)(cols / 128), (unsigned)(rows / 128)), kThreads, 0,
+                      stream, q, sf, rows, (int)cols, qt, sft) == cudaSuccess
+             ? FP8Q_OK
+             : FP8Q_ERR_CUDA;
 }
 
 }  // namespace fp8q

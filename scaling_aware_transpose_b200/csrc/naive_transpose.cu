@@ -20,6 +20,8 @@ namespace {
 __global__ void __launch_bounds__(256) dequant_kernel(const uint4* __restrict__ q, const uint8_t* __restrict__ sf,
                                                       int64_t rows, int cols, const int32_t* __restrict__ offsets,
                                                       int num_groups, uint4* __restrict__ v, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t valid_rows =
       offsets ? grouped_rows(offsets, num_groups, rows, blockIdx.x == 0 && threadIdx.x == 0 ? status : nullptr) : rows;
   if (offsets != nullptr && blockIdx.x == 0) validate_groups_cta(offsets, num_groups, status);
@@ -58,6 +60,8 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __r
                                                              const int32_t* __restrict__ offsets, int num_groups,
                                                              uint16_t* __restrict__ vt, int* status) {
   __shared__ uint16_t tile[kT][kT + kPad];
+  pdl_wait();
+  pdl_trigger();
   const int64_t valid_rows = offsets ? grouped_rows(offsets, num_groups, rows, nullptr) : rows;
   const int64_t r0 = (int64_t)blockIdx.y * kT;
   const int h0 = blockIdx.x * kT;
@@ -100,13 +104,14 @@ fp8q_status launch_naive_transpose(const DeviceInfo& dev, const uint8_t* q, cons
   uint16_t* v = static_cast<uint16_t*>(workspace);
   uint16_t* vt = v + rows * cols;
   const int64_t n16 = rows * cols / 16;
-  dequant_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, stream>>>(reinterpret_cast<const uint4*>(q), sf, rows,
-                                                                    (int)cols, offsets, num_groups,
-                                                                    reinterpret_cast<uint4*>(v), dev.status);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
-  dim3 grid((unsigned)(cols / kT), (unsigned)((rows + kT - 1) / kT));
-  transpose_bf16_kernel<<<grid, 256, 0, stream>>>(v, rows, (int)cols, offsets, num_groups, vt, dev.status);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (launch_after(dequant_kernel, dim3((unsigned)((n16 + 255) / 256)), 256, 0, stream,
+                   reinterpret_cast<const uint4*>(q), sf, rows, (int)cols, offsets, (int)num_groups,
+                   reinterpret_cast<uint4*>(v), dev.status) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  const dim3 grid((unsigned)(cols / kT), (unsigned)((rows + kT - 1) / kT));
+  if (launch_after(transpose_bf16_kernel, grid, 256, 0, stream, (const uint16_t*)v, rows, (int)cols, offsets,
+                   (int)num_groups, vt, dev.status) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
   // (3) requantize the valid part of the transposed buffer; for groups the row count
   // lives on the device (offsets[num_groups]) and the kernel reads it there.
   if (launch_quantize_tiles(vt, rows * cols / 128, qt, sft, stream, offsets ? offsets + num_groups : nullptr,

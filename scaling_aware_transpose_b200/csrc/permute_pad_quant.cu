@@ -28,6 +28,7 @@ namespace {
 __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
                                                     bool allow_drop, int32_t* __restrict__ counts, int* status) {
   extern __shared__ int32_t hist[];
+  pdl_wait();
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -468,8 +469,9 @@ fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx,
   int32_t* bases = counts + C * E;
   int32_t* totals = bases + C * E;
   const size_t hist_smem = (size_t)E * sizeof(int32_t);
-  count_kernel<<<(unsigned)C, 256, hist_smem, stream>>>(idx, npairs, E, allow_drop, counts, dev.status);
-  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (launch_after(count_kernel, dim3((unsigned)C), 256, hist_smem, stream, idx, npairs, (int)E, allow_drop, counts,
+                   dev.status) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
   // Small routings (at most 32 count loads per lane in the fused kernel's reduction) fold
   // the one-CTA scan into the rank kernel: one dependent launch fewer.
   if (E <= kRankMultiMaxE && (int64_t)((E + kRankWarps - 1) / kRankWarps) * ((C + 31) / 32) <= 32) {

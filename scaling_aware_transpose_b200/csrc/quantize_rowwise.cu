@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiles_kernel(const uint4* 
                                                                     uint8_t* __restrict__ sf, int64_t n_tiles,
                                                                     const int32_t* __restrict__ limit_rows,
                                                                     int64_t tiles_per_row) {
+  pdl_wait();
+  pdl_trigger();
   if (limit_rows != nullptr) {
     const int64_t lim = (int64_t)__ldg(limit_rows);
     n_tiles = lim <= 0 ? 0 : min(n_tiles, lim * tiles_per_row);
@@ -74,10 +76,9 @@ cudaError_t launch_quantize_tiles(const void* x, int64_t n_tiles, uint8_t* q, ui
   const int64_t tiles_per_block = (kQThreads / 32) * kQUnroll * kTilesPerWarp;
   const int64_t blocks = (n_tiles + tiles_per_block - 1) / tiles_per_block;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  quantize_tiles_kernel<<<(unsigned)blocks, kQThreads, 0, stream>>>(static_cast<const uint4*>(x),
-                                                                      reinterpret_cast<uint2*>(q), sf, n_tiles,
-                                                                      limit_rows, tiles_per_row);
-  return cudaGetLastError();
+  return launch_after(quantize_tiles_kernel, dim3((unsigned)blocks), kQThreads, 0, stream,
+                      static_cast<const uint4*>(x), reinterpret_cast<uint2*>(q), sf, n_tiles, limit_rows,
+                      tiles_per_row);
 }
 
 }  // namespace fp8q

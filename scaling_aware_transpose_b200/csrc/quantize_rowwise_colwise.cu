@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(kThreads, 4)
                                     uint8_t* __restrict__ sft) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const int64_t b = (int64_t)blockIdx.x / ncb;             // row block
@@ -175,12 +177,13 @@ fp8q_status launch_quantize_rowwise_colwise(const DeviceInfo& dev, const void* x
   if (gx * (cols / 128) > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const int zero_e = (flags & FP8Q_ZERO_TILE_MIN_SCALE) ? -127 : 0;
   const bool packed = (flags & FP8Q_SF_PACKED_UE8M0) != 0;
-  dim3 grid((unsigned)(gx * (cols / 128)));
+  const dim3 grid((unsigned)(gx * (cols / 128)));
   auto kernel = qt ? (packed ? quantize_rowwise_colwise_kernel<true, true> : quantize_rowwise_colwise_kernel<true, false>)
                    : (packed ? quantize_rowwise_colwise_kernel<false, true> : quantize_rowwise_colwise_kernel<false, false>);
-  kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(x), rows, (int)cols, zero_e, q,
-                                        static_cast<uint8_t*>(sf), qt, static_cast<uint8_t*>(sft));
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  return launch_after(kernel, grid, kThreads, 0, stream, static_cast<const uint16_t*>(x), rows, (int)cols, zero_e, q,
+                      static_cast<uint8_t*>(sf), qt, static_cast<uint8_t*>(sft)) == cudaSuccess
+             ? FP8Q_OK
+             : FP8Q_ERR_CUDA;
 }
 
 }  // namespace fp8q

@@ -25,18 +25,21 @@
 //   g >= 89:  exp(-g) <= 2^-24, 1 + exp(-g) rounds to 1, silu(g) = g (true from 16.75 on);
 //   g <= -89: exp(-g) = +inf (the exp clamp), silu(g) = g / inf = -0;
 // the last two together are max(g, -0).  The 2 x 3825 values in between are computed by
-// the spec itself into a shared-memory table at the start of each CTA, and the element
-// loop looks them up: both BF16 values of a word at once (their magnitudes clamped into
-// the range with 16-bit-lane min/max, the sign picking the half of the table), with a
-// warp vote sending the rare warp that saw an input outside the range through the
-// closed forms.  The CTAs are persistent (two per SM), so the table costs a few
-// microseconds per launch while the lookup replaces ~40 instructions per element (the
-// exp, the IEEE divide); every value is still the spec's, bit for bit.
+// the spec itself into a shared-memory table, and the element loop looks them up: both
+// BF16 values of a word at once (their magnitudes clamped into the range with 16-bit-lane
+// min/max, the sign picking the half of the table), with a warp vote sending the rare
+// warp that saw an input outside the range through the closed forms.  The lookup
+// replaces ~40 instructions per element (the exp, the IEEE divide); every value is still
+// the spec's, bit for bit.  The table is evaluated once per device: CTA 0 of the first
+// launch that finds no published table writes the one it computed to device memory and
+// then sets a ready word (release); every CTA that reads the word as set (acquire) copies
+// the 31 KB from there (L2) instead of evaluating the spec again.
 //
-// Block loop: CTA i takes blocks i, i + gridDim.x, ... (column blocks fastest).  Each
-// thread holds its 4 passes of gate/up in registers and refills a pass with the next
-// block's data as soon as it has consumed it, so three passes of loads are in flight
-// while it computes.
+// Block loop: three persistent 256-thread CTAs per SM (80 registers a thread); CTA i takes
+// blocks i, i + gridDim.x, ... (column blocks fastest).  A block is four passes of 32 rows;
+// each thread holds two passes of gate/up in registers and, as it consumes one, loads the
+// pass two ahead (crossing into its next block), so one pass of loads is in flight per
+// thread while it computes the other.
 #include "common.cuh"
 #include "launch.h"
 
@@ -87,6 +90,7 @@ constexpr uint32_t kSiluHi = 0x42B2u;  // 89
 constexpr uint32_t kTabN = kSiluHi - kSiluLo;
 constexpr uint32_t kNegBase = 4096;
 constexpr int kTab = (int)(kNegBase + kTabN);
+constexpr int kTabPad = (kTab + 3) & ~3;  // whole 16-byte pieces
 
 __device__ __forceinline__ void build_silu_table(float* tab) {
   for (int i = threadIdx.x; i < kTab; i += blockDim.x) {
@@ -94,6 +98,43 @@ __device__ __forceinline__ void build_silu_table(float* tab) {
     if (ui >= kTabN && ui < kNegBase) continue;  // unused gap
     const uint32_t h = ui < kTabN ? kSiluLo + ui : 0x8000u | (kSiluLo + ui - kNegBase);
     tab[i] = silu_spec(__uint_as_float(h << 16));
+  }
+}
+
+// The device's copy of the table and its ready word (zero until the table is published).
+__device__ __align__(16) float g_silu_tab[kTabPad];
+__device__ uint32_t g_silu_ready;
+constexpr uint32_t kSiluReady = 0x5117AB1Eu;
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Fills the CTA's table (kTabPad floats of shared memory): copied from device memory when
+// every thread's acquire load sees the ready word, else evaluated here; CTA 0 then
+// publishes it (all entries written and fenced before the release store).  Concurrent
+// first launches may publish at once; they write identical values.  Ends with a barrier.
+__device__ __forceinline__ void fill_silu_table(float* tab) {
+  const bool ready = ld_acquire_gpu(&g_silu_ready) == kSiluReady;
+  if (__syncthreads_and(ready)) {
+    const uint4* src = reinterpret_cast<const uint4*>(g_silu_tab);
+    uint4* dst = reinterpret_cast<uint4*>(tab);
+    for (int i = threadIdx.x; i < kTabPad / 4; i += blockDim.x) dst[i] = src[i];
+    __syncthreads();
+    return;
+  }
+  build_silu_table(tab);
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < kTab; i += blockDim.x) g_silu_tab[i] = tab[i];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) st_release_gpu(&g_silu_ready, kSiluReady);
   }
 }
 
@@ -114,14 +155,16 @@ __device__ __forceinline__ float sel_f32(bool p, float a, float b) {
 }
 
 // Both BF16 values of a word at once: magnitudes clamped into the table's range (16-bit
-// lanes), the sign adding 4096 to the index.  acc collects any clamped-away bits.
+// lanes), then one byte offset per lane, 4 * (magnitude - kSiluLo) + 4 * 4096 * sign (at
+// most 31680, so neither lane carries into the other).  acc collects any clamped-away bits.
 __device__ __forceinline__ void silu_lookup2(const float* tab, uint32_t w, float& lo, float& hi, uint32_t& acc) {
   const uint32_t m2 = w & 0x7FFF7FFFu;
   const uint32_t c2 = umin16x2(umax16x2(m2, kSiluLo * 0x10001u), (kSiluHi - 1) * 0x10001u);
   acc |= m2 ^ c2;
-  const uint32_t key2 = c2 + ((w >> 3) & 0x10001000u);
-  lo = tab[(key2 & 0xFFFFu) - kSiluLo];
-  hi = tab[(key2 >> 16) - kSiluLo];
+  const uint32_t off2 = ((c2 - kSiluLo * 0x10001u) << 2) + ((w >> 1) & 0x40004000u);
+  const char* tb = reinterpret_cast<const char*>(tab);
+  lo = *reinterpret_cast<const float*>(tb + (off2 & 0xFFFFu));
+  hi = *reinterpret_cast<const float*>(tb + (off2 >> 16));
 }
 
 __device__ __forceinline__ float silu_fix(float v, uint32_t h, float g) {
@@ -132,27 +175,29 @@ __device__ __forceinline__ float silu_fix(float v, uint32_t h, float g) {
 
 constexpr int kThreads = 256;
 constexpr int kPasses = 4;  // 4 passes x 32 rows x (8 threads x 16 elements)
-constexpr int kMinBlocks = 2;
+constexpr int kDepth = 2;   // passes held in registers
+constexpr int kMinBlocks = 3;
 
 __device__ __forceinline__ uint32_t swizzled_chunk(int row, int chunk) { return (uint32_t)(chunk ^ ((row >> 2) & 7)); }
 
 struct BlockIn {
-  uint4 g[kPasses][2], u[kPasses][2];
+  uint4 g[kDepth][2], u[kDepth][2];
 };
 
-// gate/up of pass p (rows p*32 + rsub) of one 128x128 block: 16 elements per thread.
+// gate/up of pass p (rows p*32 + rsub) of one 128x128 block, 16 elements per thread, into
+// register slot p % kDepth.
 __device__ __forceinline__ void load_pass(BlockIn& in, int p, const uint16_t* __restrict__ gate,
                                           const uint16_t* __restrict__ up, int64_t rows, int cols, int64_t r0, int c0,
                                           int rsub, int sub) {
   const int64_t r = r0 + p * 32 + rsub;
   if (r < rows) {
     const int64_t base = r * cols + c0 + sub * 16;
-    in.g[p][0] = ld_stream(reinterpret_cast<const uint4*>(gate + base));
-    in.g[p][1] = ld_stream(reinterpret_cast<const uint4*>(gate + base + 8));
-    in.u[p][0] = ld_stream(reinterpret_cast<const uint4*>(up + base));
-    in.u[p][1] = ld_stream(reinterpret_cast<const uint4*>(up + base + 8));
+    in.g[p % kDepth][0] = ld_stream(reinterpret_cast<const uint4*>(gate + base));
+    in.g[p % kDepth][1] = ld_stream(reinterpret_cast<const uint4*>(gate + base + 8));
+    in.u[p % kDepth][0] = ld_stream(reinterpret_cast<const uint4*>(up + base));
+    in.u[p % kDepth][1] = ld_stream(reinterpret_cast<const uint4*>(up + base + 8));
   } else {
-    in.g[p][0] = in.g[p][1] = in.u[p][0] = in.u[p][1] = make_uint4(0u, 0u, 0u, 0u);
+    in.g[p % kDepth][0] = in.g[p % kDepth][1] = in.u[p % kDepth][0] = in.u[p % kDepth][1] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -162,10 +207,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
                                                                          uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                                                                          uint8_t* __restrict__ qt,
                                                                          uint8_t* __restrict__ sft) {
-  __shared__ float silu_tab[kTab];
+  __shared__ __align__(16) float silu_tab[kTabPad];
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
   __shared__ int e_max_sh;
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
   const int sub = tid & 7;      // 16-element chunk of the row tile
@@ -174,10 +221,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
   int blk = blockIdx.x;
   BlockIn in;
 #pragma unroll
-  for (int p = 0; p < kPasses; ++p)
+  for (int p = 0; p < kDepth; ++p)
     load_pass(in, p, gate, up, rows, cols, (int64_t)(blk / ncb) * 128, (blk % ncb) * 128, rsub, sub);
-  build_silu_table(silu_tab);
-  __syncthreads();
+  fill_silu_table(silu_tab);
   for (;;) {
     const int64_t r0 = (int64_t)(blk / ncb) * 128;
     const int c0 = (blk % ncb) * 128;
@@ -190,10 +236,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
       const int rl = p * 32 + rsub;
       const int64_t r = r0 + rl;
       float y[16];
-      const uint32_t gw[8] = {in.g[p][0].x, in.g[p][0].y, in.g[p][0].z, in.g[p][0].w,
-                              in.g[p][1].x, in.g[p][1].y, in.g[p][1].z, in.g[p][1].w};
-      const uint32_t uw[8] = {in.u[p][0].x, in.u[p][0].y, in.u[p][0].z, in.u[p][0].w,
-                              in.u[p][1].x, in.u[p][1].y, in.u[p][1].z, in.u[p][1].w};
+      const int bi = p % kDepth;
+      const uint32_t gw[8] = {in.g[bi][0].x, in.g[bi][0].y, in.g[bi][0].z, in.g[bi][0].w,
+                              in.g[bi][1].x, in.g[bi][1].y, in.g[bi][1].z, in.g[bi][1].w};
+      const uint32_t uw[8] = {in.u[bi][0].x, in.u[bi][0].y, in.u[bi][0].z, in.u[bi][0].w,
+                              in.u[bi][1].x, in.u[bi][1].y, in.u[bi][1].z, in.u[bi][1].w};
       uint32_t acc = 0;
 #pragma unroll
       for (int k = 0; k < 8; ++k) silu_lookup2(silu_tab, gw[k], y[2 * k], y[2 * k + 1], acc);
@@ -228,7 +275,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
         *reinterpret_cast<uint4*>(tile + rl * 128 + (swizzled_chunk(rl, sub) << 4)) = codes;
         if (sub == 0) e_row[rl] = (uint8_t)(e + 127);
       }
-      if (next < nblk) load_pass(in, p, gate, up, rows, cols, nr0, nc0, rsub, sub);  // refill as consumed
+      if (p + kDepth < kPasses)  // refill the slot just consumed, kDepth passes ahead
+        load_pass(in, p + kDepth, gate, up, rows, cols, r0, c0, rsub, sub);
+      else if (next < nblk)
+        load_pass(in, p + kDepth - kPasses, gate, up, rows, cols, nr0, nc0, rsub, sub);
     }
 
     if (qt != nullptr) {  // uniform across the CTA
@@ -286,14 +336,14 @@ __global__ void swiglu_spec_kernel(const float* __restrict__ g, const float* __r
     y[i] = swiglu_spec(g[i], u[i]);
 }
 
-// Test hook: silu of BF16 inputs through the kernel's own table path (word-pair lookup,
-// warp vote, closed forms), for an exhaustive check against the CPU spec.  Each warp
+// Test hook: silu of BF16 inputs through the kernel's own table path (the same table fill,
+// so the device's published table once there is one; word-pair lookup, warp vote, closed
+// forms), for an exhaustive check against the CPU spec.  Each warp
 // takes 32 consecutive words per step; lanes past the end look up 1.0 (inside the table).
 __global__ void __launch_bounds__(kThreads) silu_table_kernel(const uint32_t* __restrict__ g2, int64_t nwords,
                                                               float2* __restrict__ out) {
-  __shared__ float silu_tab[kTab];
-  build_silu_table(silu_tab);
-  __syncthreads();
+  __shared__ __align__(16) float silu_tab[kTabPad];
+  fill_silu_table(silu_tab);
   const int lane = threadIdx.x & 31;
   const int64_t step = (int64_t)gridDim.x * kThreads;
   for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x - lane; base < nwords; base += step) {
@@ -319,10 +369,10 @@ fp8q_status launch_swiglu_quant(const DeviceInfo& dev, const void* gate, const v
   if (nblk > 0x7FFFFFFF - 0x10000) return FP8Q_ERR_SHAPE;  // block indices are int32
   const int64_t slots = (int64_t)dev.num_sms * kMinBlocks;
   const int64_t grid = nblk < slots ? nblk : slots;
-  swiglu_quant_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(gate),
-                                                               static_cast<const uint16_t*>(up), rows, (int)cols,
-                                                               (int)nblk, q, sf, qt, sft);
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  return launch_after(swiglu_quant_kernel, dim3((unsigned)grid), kThreads, 0, stream, static_cast<const uint16_t*>(gate),
+                      static_cast<const uint16_t*>(up), rows, (int)cols, (int)nblk, q, sf, qt, sft) == cudaSuccess
+             ? FP8Q_OK
+             : FP8Q_ERR_CUDA;
 }
 
 fp8q_status launch_debug_exp_spec_range(uint32_t first, int64_t n, float* out, cudaStream_t stream) {

@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
                                                                    const float* __restrict__ weights, int64_t tokens,
                                                                    int topk, uint16_t* __restrict__ out,
                                                                    int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int nch = hidden >> 4;
   const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (gid >= tokens * nch) return;
@@ -219,6 +221,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) unpermute_fp8_ring(const uint
                                                                       int64_t tokens, uint16_t* __restrict__ out,
                                                                       int* status) {
   extern __shared__ __align__(128) uint8_t smem[];
+  pdl_wait();
+  pdl_trigger();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // stage filled: 32 async arrivals + 1 expect-tx arrival
   uint64_t* empty = full + kRingStages;                 // stage released: one arrival per consumer warp
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kRingStages);
@@ -372,18 +376,17 @@ struct UnpermuteArgs {
 };
 
 template <bool kFp8, int kK>
-void launch_k(const UnpermuteArgs& a, unsigned blocks, cudaStream_t stream) {
-  unpermute_unpad_kernel<kFp8, kK><<<blocks, kThreads, 0, stream>>>(a.y, a.y_sf, a.rows, a.hidden, a.row_id_map,
-                                                                    a.weights, a.tokens, a.topk, a.out, a.status);
+cudaError_t launch_k(const UnpermuteArgs& a, unsigned blocks, cudaStream_t stream) {
+  return launch_after(unpermute_unpad_kernel<kFp8, kK>, dim3(blocks), kThreads, 0, stream, a.y, a.y_sf, a.rows,
+                      a.hidden, a.row_id_map, a.weights, a.tokens, a.topk, a.out, a.status);
 }
 
 template <int kK>
 cudaError_t launch_ring(const UnpermuteArgs& a, int grid, int smem, cudaStream_t stream) {
   const cudaError_t e = cudaFuncSetAttribute(unpermute_fp8_ring<kK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  unpermute_fp8_ring<kK><<<grid, kRingThreads, smem, stream>>>(a.y, a.y_sf, a.rows, a.hidden, a.row_id_map, a.weights,
-                                                               a.tokens, a.out, a.status);
-  return cudaGetLastError();
+  return launch_after(unpermute_fp8_ring<kK>, dim3((unsigned)grid), kRingThreads, (size_t)smem, stream, a.y, a.y_sf,
+                      a.rows, a.hidden, a.row_id_map, a.weights, a.tokens, a.out, a.status);
 }
 
 }  // namespace
@@ -415,22 +418,23 @@ fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const u
     }
     return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
   }
+  cudaError_t e = cudaSuccess;
   if (y_sf == nullptr) {
-    launch_k<false, 0>(a, blocks, stream);
+    e = launch_k<false, 0>(a, blocks, stream);
   } else {
     switch (topk) {
-      case 1: launch_k<true, 1>(a, blocks, stream); break;
-      case 2: launch_k<true, 2>(a, blocks, stream); break;
-      case 3: launch_k<true, 3>(a, blocks, stream); break;
-      case 4: launch_k<true, 4>(a, blocks, stream); break;
-      case 5: launch_k<true, 5>(a, blocks, stream); break;
-      case 6: launch_k<true, 6>(a, blocks, stream); break;
-      case 7: launch_k<true, 7>(a, blocks, stream); break;
-      case 8: launch_k<true, 8>(a, blocks, stream); break;
-      default: launch_k<true, 0>(a, blocks, stream); break;
+      case 1: e = launch_k<true, 1>(a, blocks, stream); break;
+      case 2: e = launch_k<true, 2>(a, blocks, stream); break;
+      case 3: e = launch_k<true, 3>(a, blocks, stream); break;
+      case 4: e = launch_k<true, 4>(a, blocks, stream); break;
+      case 5: e = launch_k<true, 5>(a, blocks, stream); break;
+      case 6: e = launch_k<true, 6>(a, blocks, stream); break;
+      case 7: e = launch_k<true, 7>(a, blocks, stream); break;
+      case 8: e = launch_k<true, 8>(a, blocks, stream); break;
+      default: e = launch_k<true, 0>(a, blocks, stream); break;
     }
   }
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 }  // namespace fp8q
