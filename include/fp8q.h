@@ -127,6 +127,8 @@ fp8q_status fp8q_naive_transpose(const uint8_t *q, const uint8_t *sf, int64_t ro
  *   q, sf    : out, as fp8q_quantize_rowwise.
  *   qt, sft  : out, [cols, rows] and [cols, rows/128], or both NULL to skip; when given,
  *              rows % 128 == 0.
+ * The first call on a device evaluates the spec's silu values once and keeps them in
+ * the library's static device memory (31 KB); later calls copy them from there.
  * Errors: NULL, ALIGN, SHAPE, ARG (only one of qt/sft given), CUDA. */
 fp8q_status fp8q_swiglu_quant(const void *gate, const void *up, int64_t rows, int64_t cols, uint8_t *q,
                               uint8_t *sf, uint8_t *qt, uint8_t *sft, fp8q_stream_t stream);
@@ -363,8 +365,8 @@ fp8q_status fp8q_debug_expire_wait(uint64_t timeout_ns, fp8q_stream_t stream);
  *     out (the value fp8q_swiglu_quant quantizes).
  *   fp8q_debug_silu_bf16: y[i] = silu(gate[i]) for n BF16 gate values (n even, gate
  *     4-byte and y 8-byte aligned), computed the way fp8q_swiglu_quant computes it (the
- *     spec's values tabulated in shared memory, looked up, closed forms outside the
- *     table's range).
+ *     spec's values tabulated in shared memory, from the device's published copy once
+ *     one exists, looked up, closed forms outside the table's range).
  * Device pointers; float arrays 4-byte aligned.  Errors: ARG, NULL, ALIGN, CUDA. */
 fp8q_status fp8q_debug_e4m3_encode_range(uint32_t first_bits, int64_t n, uint8_t *out, fp8q_stream_t stream);
 fp8q_status fp8q_debug_exp_spec_range(uint32_t first_bits, int64_t n, float *out, fp8q_stream_t stream);

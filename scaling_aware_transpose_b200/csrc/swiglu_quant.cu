@@ -173,6 +173,18 @@ __device__ __forceinline__ float silu_fix(float v, uint32_t h, float g) {
   return sel_f32(d < kTabN, v, out);
 }
 
+// max(|a|, |b|, |c|) in one instruction.
+__device__ __forceinline__ float max3abs(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// (x0, x1) *= (m0, m1): two IEEE round-to-nearest products in one packed instruction.
+__device__ __forceinline__ void mul2_rn(float& x0, float& x1, float m0, float m1) {
+  asm("{.reg .b64 x, m; mov.b64 x, {%0, %1}; mov.b64 m, {%2, %3}; mul.rn.f32x2 x, x, m; mov.b64 {%0, %1}, x;}"
+      : "+f"(x0), "+f"(x1) : "f"(m0), "f"(m1));
+}
+
 constexpr int kThreads = 256;
 constexpr int kPasses = 4;  // 4 passes x 32 rows x (8 threads x 16 elements)
 constexpr int kDepth = 2;   // passes held in registers
@@ -251,22 +263,26 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
           y[2 * k + 1] = silu_fix(y[2 * k + 1], gw[k] >> 16, __uint_as_float(gw[k] & 0xFFFF0000u));
         }
       }
-      float amax = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        y[2 * k] = __fmul_rn(y[2 * k], __uint_as_float(uw[k] << 16));
-        y[2 * k + 1] = __fmul_rn(y[2 * k + 1], __uint_as_float(uw[k] & 0xFFFF0000u));
-        amax = fmaxf(amax, fmaxf(fabsf(y[2 * k]), fabsf(y[2 * k + 1])));  // finite y: plain magnitude max
+      for (int k = 0; k < 8; ++k)  // y = silu(g) * u
+        mul2_rn(y[2 * k], y[2 * k + 1], __uint_as_float(uw[k] << 16), __uint_as_float(uw[k] & 0xFFFF0000u));
+      float amax;  // finite y: the largest magnitude, by three-input max instructions
+      {
+        const float a0 = max3abs(y[0], y[1], y[2]), a1 = max3abs(y[3], y[4], y[5]), a2 = max3abs(y[6], y[7], y[8]);
+        const float a3 = max3abs(y[9], y[10], y[11]), a4 = max3abs(y[12], y[13], y[14]);
+        amax = fmaxf(max3abs(a0, a1, a2), max3abs(a3, a4, y[15]));
       }
 #pragma unroll
       for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
       const int e = tile_exponent(amax);
       const float s = exp2_neg(e);
       uint4 codes;
-      codes.x = cvt_e4m3x2_f32(y[0] * s, y[1] * s) | (cvt_e4m3x2_f32(y[2] * s, y[3] * s) << 16);
-      codes.y = cvt_e4m3x2_f32(y[4] * s, y[5] * s) | (cvt_e4m3x2_f32(y[6] * s, y[7] * s) << 16);
-      codes.z = cvt_e4m3x2_f32(y[8] * s, y[9] * s) | (cvt_e4m3x2_f32(y[10] * s, y[11] * s) << 16);
-      codes.w = cvt_e4m3x2_f32(y[12] * s, y[13] * s) | (cvt_e4m3x2_f32(y[14] * s, y[15] * s) << 16);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mul2_rn(y[2 * k], y[2 * k + 1], s, s);
+      codes.x = cvt_e4m3x2_f32(y[0], y[1]) | (cvt_e4m3x2_f32(y[2], y[3]) << 16);
+      codes.y = cvt_e4m3x2_f32(y[4], y[5]) | (cvt_e4m3x2_f32(y[6], y[7]) << 16);
+      codes.z = cvt_e4m3x2_f32(y[8], y[9]) | (cvt_e4m3x2_f32(y[10], y[11]) << 16);
+      codes.w = cvt_e4m3x2_f32(y[12], y[13]) | (cvt_e4m3x2_f32(y[14], y[15]) << 16);
       if (r < rows) {
         *reinterpret_cast<uint4*>(q + r * cols + c0 + sub * 16) = codes;
         if (sub == 0) sf[r * ncb + (c0 >> 7)] = (uint8_t)(e + 127);
