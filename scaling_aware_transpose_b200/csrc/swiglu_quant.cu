@@ -131,7 +131,8 @@ __device__ __forceinline__ void fill_silu_table(float* tab) {
   build_silu_table(tab);
   __syncthreads();
   if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < kTab; i += blockDim.x) g_silu_tab[i] = tab[i];
+    for (int i = threadIdx.x; i < kTab; i += blockDim.x)
+      if ((uint32_t)i < kTabN || (uint32_t)i >= kNegBase) g_silu_tab[i] = tab[i];  // the gap stays zero
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) st_release_gpu(&g_silu_ready, kSiluReady);

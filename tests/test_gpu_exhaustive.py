@@ -73,7 +73,9 @@ def test_silu_table_path_matches_oracle_on_every_finite_bf16(order):
     """The fused SwiGLU kernel tabulates silu for BF16 inputs and uses closed forms outside
     the table's range; every finite BF16 gate value must give the spec's fp32 silu(g).
     Sorted, the range edges fall inside warps; shuffled, most warps that see an input
-    outside the range see only one; ragged leaves the last warp partly empty."""
+    outside the range see only one; ragged leaves the last warp partly empty.  The hook
+    fills its table the way the fused kernel does: the first call on the device evaluates
+    it and publishes it, later calls copy the published one; two calls cover both."""
     bits = np.arange(1 << 16, dtype=np.uint32)
     bits = bits[(bits & 0x7F80) != 0x7F80].astype(np.uint16)  # finite only
     if order == "shuffled":
@@ -81,11 +83,12 @@ def test_silu_table_path_matches_oracle_on_every_finite_bf16(order):
     if order == "ragged":
         bits = bits[: 2 * 1000 + 2 * 17]
     g = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
-    y = torch.empty(bits.size, dtype=torch.float32, device="cuda")
-    sat.fp8q_debug_silu_bf16(g, bits.size, y)
-    got = y.cpu().numpy().view(np.uint32)
     gf = (bits.astype(np.uint32) << 16).view(np.float32)
     want = oracle.swiglu(gf, np.ones_like(gf)).view(np.uint32)   # silu(g) * 1
-    bad = np.flatnonzero(got != want)
-    assert bad.size == 0, (f"{bad.size} of {bits.size} differ; first g bits {hex(int(bits[bad[0]]))}: "
-                           f"got {hex(got[bad[0]])} want {hex(want[bad[0]])}")
+    for call in range(2):
+        y = torch.full((bits.size,), float("nan"), dtype=torch.float32, device="cuda")
+        sat.fp8q_debug_silu_bf16(g, bits.size, y)
+        got = y.cpu().numpy().view(np.uint32)
+        bad = np.flatnonzero(got != want)
+        assert bad.size == 0, (f"call {call}: {bad.size} of {bits.size} differ; first g bits "
+                               f"{hex(int(bits[bad[0]]))}: got {hex(got[bad[0]])} want {hex(want[bad[0]])}")
