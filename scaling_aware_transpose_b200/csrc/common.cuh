@@ -28,8 +28,25 @@ __device__ __forceinline__ void record_status(int* status, int code) { atomicCAS
 // chain (routing -> payload) a kernel may trigger early and wait only where it first
 // reads its predecessor's output.  In a launch without the attribute, or after a kernel
 // that never triggers, both are no-ops and the launch is ordered as usual.
+//
+// The wait orders memory accesses only if the compiler keeps them after it.  A load the
+// compiler may treat as invariant (a plain load through a const __restrict__ pointer it
+// turns into a read-only one) is free to move above an asm statement, so every load after
+// a wait goes through a pointer passed through pdl_wait_for(): each pointer becomes the
+// output of an empty volatile asm placed after the wait, a value the compiler cannot see
+// through, and every address formed from it depends on that output.  (The read-only path
+// itself is not used at all; see ld_g.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+template <typename P>
+__device__ __forceinline__ void make_opaque(P& p) {  // p: any pointer variable
+  asm volatile("" : "+l"(p));
+}
+template <typename... P>
+__device__ __forceinline__ void pdl_wait_for(P&... ptrs) {
+  pdl_wait();
+  (make_opaque(ptrs), ...);
+}
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, unsigned block, size_t smem, cudaStream_t stream,
@@ -278,6 +295,15 @@ __device__ __forceinline__ int64_t grouped_rows(const int32_t* off, int G, int64
 }
 
 // ------------------------------------------------------------------ memory
+// Global loads are ordinary coherent loads (ld_g) or evict-first ones (ld_stream), never
+// the read-only path (ld.global.nc, __ldg): with dependent launches a kernel's lifetime
+// overlaps its predecessor's, which may still be writing what the kernel reads after its
+// wait, and the read-only path requires data that stays unchanged for the reading
+// kernel's whole lifetime.
+template <typename T>
+__device__ __forceinline__ T ld_g(const T* p) {
+  return *p;
+}
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 // 8-byte store marked evict-first (written once, not read again by this kernel).
 __device__ __forceinline__ void st_stream8(void* p, uint2 v) {

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kThreads, kGrouped ? 6 : 8) direct_transpose_k
                                                                      uint8_t* __restrict__ sft, int* status) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
-  pdl_wait();
+  pdl_wait_for(q, sf, off);
   pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
@@ -87,9 +87,9 @@ __global__ void __launch_bounds__(kThreads, kGrouped ? 6 : 8) direct_transpose_k
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
     const uint4* src = reinterpret_cast<const uint4*>(qb + (p * 32 + rsub) * cols) + sub;
-    v[p] = kGrouped ? __ldg(src) : ld_stream(src);
+    v[p] = kGrouped ? ld_g(src) : ld_stream(src);
   }
-  if (tid < 128) e_row[tid] = __ldg(sf + (r0 + tid) * ncb + j);
+  if (tid < 128) e_row[tid] = ld_g(sf + (r0 + tid) * ncb + j);
   __syncthreads();
   const uint32_t ew = reinterpret_cast<const uint32_t*>(e_row)[tid & 31];
   int m = (int)max(max(ew & 0xFFu, (ew >> 8) & 0xFFu), max((ew >> 16) & 0xFFu, ew >> 24));
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks2x1) direct_transpose_2x1(
   __shared__ __align__(128) uint8_t tile[256 * 128];
   __shared__ __align__(16) uint8_t e_row[256];
   __shared__ int emax_w[8];
-  pdl_wait();
+  pdl_wait_for(q, sf);
   pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks2x1) direct_transpose_2x1(
     cp_async16(tile + row * 128 + 16 * chunk_pos2(row, c), qb + (int64_t)row * cols + 16 * c);
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-  const int e = __ldg(sf + (r0 + tid) * ncb + j);  // scale byte of row tid
+  const int e = ld_g(sf + (r0 + tid) * ncb + j);  // scale byte of row tid
   e_row[tid] = (uint8_t)e;
   const int lane = tid & 31, wi = tid >> 5;  // warp wi holds rows 32wi..32wi+31: row block wi >> 2
   const unsigned wm = __reduce_max_sync(0xFFFFFFFFu, (unsigned)e);

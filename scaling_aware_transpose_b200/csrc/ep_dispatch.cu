@@ -51,45 +51,59 @@ __device__ __forceinline__ int segment_of(const int64_t* start, int n, int64_t x
 }
 
 // Pair (t, d) of the send-side routing: d if some slot of token t has its expert on rank
-// d, else -1.  The d == 0 thread of each token checks the ids.
-__global__ void __launch_bounds__(256) dest_kernel(const int32_t* __restrict__ idx, int64_t tokens, int K, int W,
-                                                   int Eloc, int32_t* __restrict__ didx, int* status) {
-  pdl_wait();
+// d, else -1; the d == 0 thread of each token checks the ids.  Fused with the routing's
+// first step: each CTA takes one chunk of kChunk pairs (p = t*W + d, row-major) and also
+// writes that chunk's per-destination pair counts, the histogram layout the rank kernels
+// read (counts[chunk][d]).  One thread per pair.
+__global__ void __launch_bounds__(kChunk) dest_count_kernel(const int32_t* __restrict__ idx, int64_t tokens, int K,
+                                                             int W, int Eloc, int32_t* __restrict__ didx,
+                                                             int32_t* __restrict__ counts, int* status) {
+  extern __shared__ int32_t hist[];  // W entries
+  pdl_wait_for(idx);
   pdl_trigger();
-  const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (p >= tokens * W) return;
-  const int64_t t = p / W;
-  const int d = (int)(p - t * W);
+  for (int e = threadIdx.x; e < W; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t npairs = tokens * W;
   const int64_t E = (int64_t)W * Eloc;
-  bool hit = false, bad = false;
-  for (int k = 0; k < K; ++k) {
-    const int32_t e = __ldg(idx + t * K + k);
-    if (e < 0 || e >= E) {
-      bad = true;
-      continue;
+  const int64_t p0 = (int64_t)blockIdx.x * kChunk;
+  for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
+    const int64_t p = p0 + i;
+    if (p >= npairs) break;
+    const int64_t t = p / W;
+    const int d = (int)(p - t * W);
+    bool hit = false, bad = false;
+    for (int k = 0; k < K; ++k) {
+      const int32_t e = ld_g(idx + t * K + k);
+      if (e < 0 || e >= E) {
+        bad = true;
+        continue;
+      }
+      hit |= e / Eloc == d;
     }
-    hit |= e / Eloc == d;
+    if (bad && d == 0) record_status(status, FP8Q_ERR_DEVICE);
+    didx[p] = hit ? d : -1;
+    if (hit) atomicAdd(&hist[d], 1);
   }
-  if (bad && d == 0) record_status(status, FP8Q_ERR_DEVICE);
-  didx[p] = hit ? d : -1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < W; e += blockDim.x) counts[(int64_t)blockIdx.x * W + e] = hist[e];
 }
 
 // Slot ids of each sent row, re-expressed for its destination rank.  A dependent launch
 // after the routing: it waits for the send map before reading it.
 __global__ void __launch_bounds__(256) send_ids_kernel(const int32_t* __restrict__ idx, int64_t tokens, int K, int W,
                                                        int Eloc, const int32_t* __restrict__ send_map,
-                                                       int32_t* __restrict__ send_ids) {
+                                                       int32_t* __restrict__ send_ids, int64_t max_rows) {
   pdl_trigger();
-  pdl_wait();
+  pdl_wait_for(send_map, idx);
   const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (p >= tokens * W) return;
-  const int32_t row = send_map[p];
-  if (row < 0) return;
+  const int32_t row = ld_g(send_map + p);
+  if (row < 0 || row >= max_rows) return;  // (never out of range for a consistent routing)
   const int64_t t = p / W;
   const int d = (int)(p - t * W);
   const int64_t E = (int64_t)W * Eloc;
   for (int k = 0; k < K; ++k) {
-    const int32_t e = __ldg(idx + t * K + k);
+    const int32_t e = ld_g(idx + t * K + k);
     send_ids[(int64_t)row * K + k] = (e >= 0 && e < E && e / Eloc == d) ? e - d * Eloc : -1;
   }
 }
@@ -103,7 +117,9 @@ __global__ void __launch_bounds__(256) gather_ids_kernel(const __grid_constant__
   if (p >= npairs) return;
   const int64_t r = p / K;
   const int s = segment_of(tab.row_start, tab.n, r);
-  rid[p] = __ldg(tab.ids[s] + (r - tab.row_start[s]) * K + (p - r * K));
+  const int32_t* ids = tab.ids[s];
+  make_opaque(ids);  // after the wait (see pdl_wait_for)
+  rid[p] = ld_g(ids + (r - tab.row_start[s]) * K + (p - r * K));
 }
 
 // Payload of the receive side: the CTAs of segment s cover its tiles (row, column block)
@@ -116,11 +132,12 @@ __global__ void __launch_bounds__(kSThreads) scatter_segments_kernel(const __gri
                                                                      uint8_t* __restrict__ sf, int64_t scatter_ctas,
                                                                      int pad_slots,
                                                                      const int32_t* __restrict__ offsets,
-                                                                     const int32_t* __restrict__ totals) {
+                                                                     const int32_t* __restrict__ totals,
+                                                                     int64_t max_rows) {
   if ((int64_t)blockIdx.x >= scatter_ctas) {
-    pdl_wait();  // the offsets
+    pdl_wait_for(offsets, totals);  // the offsets
     pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
-             reinterpret_cast<uint8_t*>(q), sf);
+             reinterpret_cast<uint8_t*>(q), sf, max_rows);
     return;
   }
   const int s = segment_of(tab.cta_start, tab.n, (int64_t)blockIdx.x);
@@ -140,10 +157,10 @@ __global__ void __launch_bounds__(kSThreads) scatter_segments_kernel(const __gri
     e[u] = 0;
     if (tile[u] < n_tiles) {
       v[u] = ld_stream(xq + tile[u] * 8 + sub);
-      if (sub == 0) e[u] = __ldg(xsf + tile[u]);
+      if (sub == 0) e[u] = ld_g(xsf + tile[u]);
     }
   }
-  pdl_wait();  // the row ids
+  pdl_wait_for(row_id_map);  // the row ids
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
     if (tile[u] >= n_tiles) continue;
@@ -151,8 +168,8 @@ __global__ void __launch_bounds__(kSThreads) scatter_segments_kernel(const __gri
     const int j = (int)(tile[u] - t * ncb);
     const int32_t* ids = row_id_map + (r0 + t) * topk;
     for (int k = 0; k < topk; ++k) {
-      const int32_t row = __ldg(ids + k);
-      if (row < 0) continue;
+      const int32_t row = ld_g(ids + k);
+      if (row < 0 || row >= max_rows) continue;  // (never out of range for a consistent routing)
       q[((int64_t)row * ncb + j) * 8 + sub] = v[u];
       if (sub == 0) sf[(int64_t)row * ncb + j] = e[u];
     }
@@ -210,20 +227,21 @@ extern "C" fp8q_status fp8q_ep_dispatch_pack(const uint8_t* xq, const uint8_t* x
   int32_t* didx = static_cast<int32_t*>(workspace);
   void* route_ws = static_cast<uint8_t*>(workspace) + round16((size_t)(tokens * W) * sizeof(int32_t));
   const int64_t npairs = tokens * W;
-  if (launch_after(dest_kernel, dim3((unsigned)((npairs + 255) / 256)), 256, 0, st, topk_idx, tokens, (int)K, (int)W,
-                   (int)Eloc, didx, dev.status) != cudaSuccess)
+  if (launch_after(dest_count_kernel, dim3((unsigned)num_chunks(tokens, W)), kChunk, (size_t)W * sizeof(int32_t), st,
+                   topk_idx, tokens, (int)K, (int)W, (int)Eloc, didx, static_cast<int32_t*>(route_ws),
+                   dev.status) != cudaSuccess)
     return FP8Q_ERR_CUDA;
-  fp8q_status rs = route_pairs(dev, tokens, didx, W, W, 1, true, send_offsets, send_map, route_ws, st);
+  fp8q_status rs = route_ranks(dev, tokens, didx, W, W, 1, send_offsets, send_map, route_ws, true, st);
   if (rs != FP8Q_OK) return rs;
   // The slot ids need only the send map; launched before the payload (both as dependent
   // launches), so the payload's loads overlap them.
   const int32_t* smap = send_map;
   if (launch_after(send_ids_kernel, (unsigned)((npairs + 255) / 256), 256, 0, st, topk_idx, tokens, K, W, Eloc, smap,
-                   send_ids) != cudaSuccess)
+                   send_ids, max_send_rows) != cudaSuccess)
     return FP8Q_ERR_CUDA;
   if (hidden > 0)
-    return launch_scatter_copy(xq, xsf, tokens, hidden, send_map, W, W, 1, send_q, send_sf, send_offsets,
-                               route_totals(route_ws, tokens, W, W), st);
+    return launch_scatter_copy(xq, xsf, tokens, hidden, send_map, W, W, 1, send_q, send_sf, max_send_rows,
+                               send_offsets, route_totals(route_ws, tokens, W, W), st);
   return FP8Q_OK;
 }
 
@@ -296,6 +314,6 @@ extern "C" fp8q_status fp8q_ep_recv_permute_fp8(const fp8q_ep_source* sources, i
   const int32_t* offs = expert_offsets;
   const int32_t* tots = route_totals(route_ws, R, K, Eloc);
   const cudaError_t rc = launch_after(scatter_segments_kernel, (unsigned)blocks, kSThreads, 0, st, tab, ncb, rmap, K,
-                                      reinterpret_cast<uint4*>(q), sf, ctas, pad_slots, offs, tots);
+                                      reinterpret_cast<uint4*>(q), sf, ctas, pad_slots, offs, tots, max_out_rows);
   return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }

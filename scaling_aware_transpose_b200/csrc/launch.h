@@ -48,13 +48,21 @@ size_t permute_workspace_bytes(int64_t tokens, int32_t topk, int32_t num_experts
 fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx, int32_t slots, int32_t E,
                         int32_t align, bool allow_drop, int32_t* offsets, int32_t* row_id_map, void* workspace,
                         cudaStream_t stream);
+// The part of route_pairs after its histogram launch, for callers whose own kernel wrote
+// the per-chunk histograms (counts[c][e] of chunk c's kChunk pairs, at the workspace's
+// start).  ids_wait: the ids were written by the kernel launched just before (the rank
+// kernels then wait for it before loading them).
+fp8q_status route_ranks(const DeviceInfo& dev, int64_t rows, const int32_t* idx, int32_t slots, int32_t E,
+                        int32_t align, int32_t* offsets, int32_t* row_id_map, void* workspace, bool ids_wait,
+                        cudaStream_t stream);
 const int32_t* route_totals(const void* workspace, int64_t rows, int32_t slots, int32_t E);
 // FP8 payload of a routing: row r's codes and scale bytes go to rows row_id_map[r*slots
 // + s] (skipped where -1); the trailing CTAs zero-fill each group's padding rows.  A
 // programmatic dependent launch: it waits for the routing kernels before reading ids.
 fp8q_status launch_scatter_copy(const uint8_t* xq, const uint8_t* xsf, int64_t rows, int64_t hidden,
                                 const int32_t* row_id_map, int32_t slots, int32_t E, int32_t align, uint8_t* q,
-                                uint8_t* sf, const int32_t* offsets, const int32_t* totals, cudaStream_t stream);
+                                uint8_t* sf, int64_t max_rows, const int32_t* offsets, const int32_t* totals,
+                                cudaStream_t stream);
 fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64_t tokens, int64_t hidden,
                                      const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
                                      uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,

@@ -39,7 +39,7 @@ __device__ __forceinline__ uint32_t chunk_maxabs(const uint4& v) {
 
 __global__ void __launch_bounds__(kQThreads) quantize_mx32_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
                                                                    uint8_t* __restrict__ sf, int64_t n_tiles) {
-  pdl_wait();
+  pdl_wait_for(x);
   pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * kQThreads + threadIdx.x) >> 5;
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ uint32_t e_row[128];  // 4 scale bytes of the row: column groups 0..3 of this tile
   __shared__ __align__(16) uint32_t smax_rg[4];  // row group rg: Smax byte of column groups 0..3
-  pdl_wait();
+  pdl_wait_for(q, sf);
   pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
@@ -97,12 +97,12 @@ __global__ void __launch_bounds__(kThreads, 6) direct_transpose_mx32_kernel(cons
   const uint8_t* qb = q + r0 * cols + c0;
   uint4 v[kPasses];
 #pragma unroll
-  for (int p = 0; p < kPasses; ++p) v[p] = __ldg(reinterpret_cast<const uint4*>(qb + (p * 32 + rsub) * cols) + sub);
+  for (int p = 0; p < kPasses; ++p) v[p] = ld_g(reinterpret_cast<const uint4*>(qb + (p * 32 + rsub) * cols) + sub);
   // The row's 4 scale bytes (4-byte aligned: rows of cols/32 bytes, cols % 128 == 0).
   // Warp rg < 4 loads the 32 rows of row group rg and reduces their Smax per column group
   // with single-instruction warp reductions, one packed word per row group.
   if (tid < 128) {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(sf + (r0 + tid) * ngr + (c0 >> 5)));
+    const uint32_t w = ld_g(reinterpret_cast<const uint32_t*>(sf + (r0 + tid) * ngr + (c0 >> 5)));
     e_row[tid] = w;
     uint32_t m = 0;
 #pragma unroll

@@ -20,7 +20,7 @@ namespace {
 __global__ void __launch_bounds__(256) dequant_kernel(const uint4* __restrict__ q, const uint8_t* __restrict__ sf,
                                                       int64_t rows, int cols, const int32_t* __restrict__ offsets,
                                                       int num_groups, uint4* __restrict__ v, int* status) {
-  pdl_wait();
+  pdl_wait_for(q, sf, offsets);
   pdl_trigger();
   const int64_t valid_rows =
       offsets ? grouped_rows(offsets, num_groups, rows, blockIdx.x == 0 && threadIdx.x == 0 ? status : nullptr) : rows;
@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint4* __restrict__ 
   const int64_t elem = i * 16;
   const int64_t r = elem / cols;
   const int h = (int)(elem - r * cols);
-  const int e = (int)__ldg(sf + r * (cols >> 7) + (h >> 7)) - 127;
+  const int e = (int)ld_g(sf + r * (cols >> 7) + (h >> 7)) - 127;
   // 2^e as fp32, e in [-127, 127]: 2^-127 is the subnormal 0x00400000
   const float s = e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
   const uint4 c = ld_stream(q + i);
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __r
                                                              const int32_t* __restrict__ offsets, int num_groups,
                                                              uint16_t* __restrict__ vt, int* status) {
   __shared__ uint16_t tile[kT][kT + kPad];
-  pdl_wait();
+  pdl_wait_for(v, offsets);
   pdl_trigger();
   const int64_t valid_rows = offsets ? grouped_rows(offsets, num_groups, rows, nullptr) : rows;
   const int64_t r0 = (int64_t)blockIdx.y * kT;

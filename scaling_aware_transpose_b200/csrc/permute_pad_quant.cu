@@ -28,7 +28,7 @@ namespace {
 __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
                                                     bool allow_drop, int32_t* __restrict__ counts, int* status) {
   extern __shared__ int32_t hist[];
-  pdl_wait();
+  pdl_wait_for(idx);
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ 
   for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
     const int64_t p = p0 + i;
     if (p >= npairs) break;
-    const int32_t e = __ldg(idx + p);
+    const int32_t e = ld_g(idx + p);
     if (e < 0 || e >= E) {
       if (!(allow_drop && e == -1)) record_status(status, FP8Q_ERR_DEVICE);
       continue;
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
   __shared__ int32_t s_warp[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_trigger();
-  pdl_wait();  // the histograms
+  pdl_wait_for(counts);  // the histograms
   for (int e = warp; e < E; e += 32) {
     int32_t acc = 0;
     for (int64_t c0 = 0; c0 < C; c0 += 8 * 32) {
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int64_t c = c0 + u * 32 + lane;
-        v[u] = c < C ? __ldg(counts + c * E + e) : 0;
+        v[u] = c < C ? ld_g(counts + c * E + e) : 0;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) acc += v[u];
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int64_t c = c0 + u * 32 + lane;
-        v[u] = c < C ? __ldg(counts + c * E + e) : 0;
+        v[u] = c < C ? ld_g(counts + c * E + e) : 0;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -134,18 +134,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 }
 
 __global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
-                                                  const int32_t* __restrict__ bases, int32_t* __restrict__ row_id_map) {
+                                                  const int32_t* __restrict__ bases, int32_t* __restrict__ row_id_map,
+                                                  bool ids_wait) {
   extern __shared__ int32_t run[];
   const int lane = threadIdx.x;
   const int64_t p0 = (int64_t)blockIdx.x * kChunk;
   int32_t ids[kChunk / 32];
+  if (ids_wait) pdl_wait_for(idx);  // the ids were written inside this call (see route_ranks)
 #pragma unroll
   for (int i = 0; i < kChunk / 32; ++i) {
     const int64_t p = p0 + i * 32 + lane;
-    ids[i] = p < npairs ? __ldg(idx + p) : -1;
+    ids[i] = p < npairs ? ld_g(idx + p) : -1;
   }
   pdl_trigger();
-  pdl_wait();  // the bases
+  pdl_wait_for(bases);  // the bases
   for (int e = lane; e < E; e += 32) run[e] = bases[(int64_t)blockIdx.x * E + e];
   __syncwarp();
 #pragma unroll 4
@@ -178,16 +180,17 @@ constexpr int kRankWarps = 8;
 constexpr int kRankMultiMaxE = 512;
 __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32_t* __restrict__ idx, int64_t npairs,
                                                                      int E, const int32_t* __restrict__ bases,
-                                                                     int32_t* __restrict__ row_id_map) {
+                                                                     int32_t* __restrict__ row_id_map, bool ids_wait) {
   extern __shared__ int32_t s_cnt[];  // [kRankWarps][E]
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   constexpr int kPer = kChunk / kRankWarps / 32;  // iterations per warp
   const int64_t p0 = (int64_t)blockIdx.x * kChunk + w * (kChunk / kRankWarps);
   int32_t ids[kPer];
+  if (ids_wait) pdl_wait_for(idx);  // the ids were written inside this call (see route_ranks)
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int64_t p = p0 + i * 32 + lane;
-    ids[i] = p < npairs ? __ldg(idx + p) : -1;
+    ids[i] = p < npairs ? ld_g(idx + p) : -1;
   }
   pdl_trigger();
   for (int e = tid; e < kRankWarps * E; e += blockDim.x) s_cnt[e] = 0;
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
     __syncwarp();
   }
   __syncthreads();
-  pdl_wait();  // the bases
+  pdl_wait_for(bases);  // the bases
   for (int e = tid; e < E; e += blockDim.x) {
     int32_t run = bases[(int64_t)blockIdx.x * E + e];
 #pragma unroll
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_fused_kernel(const int32
                                                                      int E, int align, const int32_t* __restrict__ counts,
                                                                      int64_t C, int32_t* __restrict__ offsets,
                                                                      int32_t* __restrict__ totals,
-                                                                     int32_t* __restrict__ row_id_map) {
+                                                                     int32_t* __restrict__ row_id_map, bool ids_wait) {
   extern __shared__ int32_t s_cnt[];  // [kRankWarps][E] | pre[E] | tot[E] | off[E] | warp sums[kRankWarps]
   int32_t* s_pre = s_cnt + kRankWarps * E;
   int32_t* s_tot = s_pre + E;
@@ -255,10 +258,11 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_fused_kernel(const int32
   constexpr int kPer = kChunk / kRankWarps / 32;
   const int64_t p0 = (int64_t)blockIdx.x * kChunk + w * (kChunk / kRankWarps);
   int32_t ids[kPer];
+  if (ids_wait) pdl_wait_for(idx);  // the ids were written inside this call (see route_ranks)
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int64_t p = p0 + i * 32 + lane;
-    ids[i] = p < npairs ? __ldg(idx + p) : -1;
+    ids[i] = p < npairs ? ld_g(idx + p) : -1;
   }
   pdl_trigger();
   for (int e = tid; e < kRankWarps * E; e += blockDim.x) s_cnt[e] = 0;
@@ -273,11 +277,11 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_fused_kernel(const int32
     if (ok && lane == __ffs(same) - 1) mine[e] += __popc(same);
     __syncwarp();
   }
-  pdl_wait();  // the histograms
+  pdl_wait_for(counts);  // the histograms
   for (int e = w; e < E; e += kRankWarps) {
     int32_t tot = 0, pre = 0;
     for (int64_t c = lane; c < C; c += 32) {
-      const int32_t v = __ldg(counts + c * E + e);
+      const int32_t v = ld_g(counts + c * E + e);
       tot += v;
       pre += c < (int64_t)blockIdx.x ? v : 0;
     }
@@ -351,11 +355,12 @@ __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* _
                                                                   uint2* __restrict__ q, uint8_t* __restrict__ sf,
                                                                   int64_t scatter_ctas, int pad_slots,
                                                                   const int32_t* __restrict__ offsets,
-                                                                  const int32_t* __restrict__ totals) {
+                                                                  const int32_t* __restrict__ totals,
+                                                                  int64_t max_rows) {
   if ((int64_t)blockIdx.x >= scatter_ctas) {
-    pdl_wait();  // the offsets
+    pdl_wait_for(offsets, totals);  // the offsets
     pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
-             reinterpret_cast<uint8_t*>(q), sf);
+             reinterpret_cast<uint8_t*>(q), sf, max_rows);
     return;
   }
   const int lane = threadIdx.x & 31, sub = lane & 7;
@@ -387,15 +392,15 @@ __global__ void __launch_bounds__(kSThreads) scatter_quant_kernel(const uint4* _
     lo[u] = make_uint2(encode4(v0[u].x, v0[u].y, s), encode4(v0[u].z, v0[u].w, s));
     hi[u] = make_uint2(encode4(v1[u].x, v1[u].y, s), encode4(v1[u].z, v1[u].w, s));
   }
-  pdl_wait();  // the row ids: everything above overlaps the routing
+  pdl_wait_for(row_id_map);  // the row ids: everything above overlaps the routing
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
     if (tile[u] >= n_tiles) continue;
     const int64_t t = tile[u] / ncb;
     const int j = (int)(tile[u] - t * ncb);
     for (int k = 0; k < topk; ++k) {
-      const int32_t row = __ldg(row_id_map + t * topk + k);
-      if (row < 0) continue;
+      const int32_t row = ld_g(row_id_map + t * topk + k);
+      if (row < 0 || row >= max_rows) continue;  // (never out of range for a consistent routing)
       uint2* dst = q + ((int64_t)row * ncb + j) * 16;
       dst[sub] = lo[u];
       dst[8 + sub] = hi[u];
@@ -414,11 +419,11 @@ __global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __
                                                                  int topk, uint4* __restrict__ q,
                                                                  uint8_t* __restrict__ sf, int64_t scatter_ctas,
                                                                  int pad_slots, const int32_t* __restrict__ offsets,
-                                                                 const int32_t* __restrict__ totals) {
+                                                                 const int32_t* __restrict__ totals, int64_t max_rows) {
   if ((int64_t)blockIdx.x >= scatter_ctas) {
-    pdl_wait();  // the offsets
+    pdl_wait_for(offsets, totals);  // the offsets
     pad_rows((int64_t)blockIdx.x - scatter_ctas, pad_slots, offsets, totals, (int64_t)ncb * 128,
-             reinterpret_cast<uint8_t*>(q), sf);
+             reinterpret_cast<uint8_t*>(q), sf, max_rows);
     return;
   }
   const int lane = threadIdx.x & 31, sub = lane & 7;
@@ -434,18 +439,18 @@ __global__ void __launch_bounds__(kSThreads) scatter_copy_kernel(const uint4* __
     e[u] = 0;
     if (tile[u] < n_tiles) {
       v[u] = ld_stream(xq + tile[u] * 8 + sub);
-      if (sub == 0) e[u] = __ldg(xsf + tile[u]);
+      if (sub == 0) e[u] = ld_g(xsf + tile[u]);
     }
   }
-  pdl_wait();  // the row ids
+  pdl_wait_for(row_id_map);  // the row ids
 #pragma unroll
   for (int u = 0; u < kSUnroll; ++u) {
     if (tile[u] >= n_tiles) continue;
     const int64_t t = tile[u] / ncb;
     const int j = (int)(tile[u] - t * ncb);
     for (int k = 0; k < topk; ++k) {
-      const int32_t row = __ldg(row_id_map + t * topk + k);
-      if (row < 0) continue;
+      const int32_t row = ld_g(row_id_map + t * topk + k);
+      if (row < 0 || row >= max_rows) continue;  // (never out of range for a consistent routing)
       q[((int64_t)row * ncb + j) * 8 + sub] = v[u];
       if (sub == 0) sf[(int64_t)row * ncb + j] = e[u];
     }
@@ -466,18 +471,34 @@ fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx,
   const int64_t npairs = rows * slots;
   const int64_t C = num_chunks(rows, slots);
   int32_t* counts = static_cast<int32_t*>(workspace);
-  int32_t* bases = counts + C * E;
-  int32_t* totals = bases + C * E;
   const size_t hist_smem = (size_t)E * sizeof(int32_t);
   if (launch_after(count_kernel, dim3((unsigned)C), 256, hist_smem, stream, idx, npairs, (int)E, allow_drop, counts,
                    dev.status) != cudaSuccess)
     return FP8Q_ERR_CUDA;
+  return route_ranks(dev, rows, idx, slots, E, align, offsets, row_id_map, workspace, false, stream);
+}
+
+// Steps (2)-(3) after the per-chunk histograms are in the workspace's counts.  The rank
+// kernels load their chunk's ids before waiting on their predecessor; that is safe when
+// the ids existed before the call (after route_pairs' histogram kernel, which waits before
+// it lets them start).  ids_wait makes them wait first, for ids written by the kernel
+// just before.
+fp8q_status route_ranks(const DeviceInfo& dev, int64_t rows, const int32_t* idx, int32_t slots, int32_t E,
+                        int32_t align, int32_t* offsets, int32_t* row_id_map, void* workspace, bool ids_wait,
+                        cudaStream_t stream) {
+  (void)dev;
+  const int64_t npairs = rows * slots;
+  const int64_t C = num_chunks(rows, slots);
+  int32_t* counts = static_cast<int32_t*>(workspace);
+  int32_t* bases = counts + C * E;
+  int32_t* totals = bases + C * E;
+  const size_t hist_smem = (size_t)E * sizeof(int32_t);
   // Small routings (at most 32 count loads per lane in the fused kernel's reduction) fold
   // the one-CTA scan into the rank kernel: one dependent launch fewer.
   if (E <= kRankMultiMaxE && (int64_t)((E + kRankWarps - 1) / kRankWarps) * ((C + 31) / 32) <= 32) {
     const size_t smem = ((size_t)(kRankWarps + 3) * E + kRankWarps) * sizeof(int32_t);
     return launch_after(rank_fused_kernel, (unsigned)C, kRankWarps * 32, smem, stream, idx, npairs, E, (int)align,
-                        (const int32_t*)counts, C, offsets, totals, row_id_map) == cudaSuccess
+                        (const int32_t*)counts, C, offsets, totals, row_id_map, ids_wait) == cudaSuccess
                ? FP8Q_OK
                : FP8Q_ERR_CUDA;
   }
@@ -487,9 +508,9 @@ fp8q_status route_pairs(const DeviceInfo& dev, int64_t rows, const int32_t* idx,
   const cudaError_t rc =
       E <= kRankMultiMaxE
           ? launch_after(rank_multi_kernel, (unsigned)C, kRankWarps * 32, (size_t)kRankWarps * E * sizeof(int32_t),
-                         stream, idx, npairs, E, (const int32_t*)bases, row_id_map)
+                         stream, idx, npairs, E, (const int32_t*)bases, row_id_map, ids_wait)
           : launch_after(rank_kernel, (unsigned)C, 32, hist_smem, stream, idx, npairs, E, (const int32_t*)bases,
-                         row_id_map);
+                         row_id_map, ids_wait);
   return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -502,8 +523,8 @@ namespace {
 // xq/xsf != nullptr: FP8-input payload; else quantize x.
 fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq, const uint8_t* xsf, int64_t tokens,
                         int64_t hidden, const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
-                        uint8_t* q, uint8_t* sf, int32_t* expert_offsets, int32_t* row_id_map, void* workspace,
-                        cudaStream_t stream) {
+                        uint8_t* q, uint8_t* sf, int64_t max_rows, int32_t* expert_offsets, int32_t* row_id_map,
+                        void* workspace, cudaStream_t stream) {
   const int E = num_experts;
   if (tokens == 0) {
     return cudaMemsetAsync(expert_offsets, 0, (size_t)(E + 1) * sizeof(int32_t), stream) == cudaSuccess
@@ -525,10 +546,11 @@ fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq,
   const int32_t* rmap = row_id_map;
   const int32_t* offs = expert_offsets;
   const int32_t* tots = totals;
-  if (xq) return launch_scatter_copy(xq, xsf, tokens, hidden, rmap, topk, E, align, q, sf, offs, tots, stream);
+  if (xq)
+    return launch_scatter_copy(xq, xsf, tokens, hidden, rmap, topk, E, align, q, sf, max_rows, offs, tots, stream);
   const cudaError_t rc = launch_after(scatter_quant_kernel, (unsigned)blocks, kSThreads, 0, stream,
                                       static_cast<const uint4*>(x), tokens, ncb, rmap, (int)topk,
-                                      reinterpret_cast<uint2*>(q), sf, scatter_ctas, pad_slots, offs, tots);
+                                      reinterpret_cast<uint2*>(q), sf, scatter_ctas, pad_slots, offs, tots, max_rows);
   return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -536,7 +558,8 @@ fp8q_status permute_pad(const DeviceInfo& dev, const void* x, const uint8_t* xq,
 
 fp8q_status launch_scatter_copy(const uint8_t* xq, const uint8_t* xsf, int64_t rows, int64_t hidden,
                                 const int32_t* row_id_map, int32_t slots, int32_t E, int32_t align, uint8_t* q,
-                                uint8_t* sf, const int32_t* offsets, const int32_t* totals, cudaStream_t stream) {
+                                uint8_t* sf, int64_t max_rows, const int32_t* offsets, const int32_t* totals,
+                                cudaStream_t stream) {
   const int ncb = (int)(hidden / 128);
   const int64_t n_tiles = rows * ncb;
   const int64_t tiles_per_block = (kSThreads / 32) * kSUnroll * 4;
@@ -546,7 +569,8 @@ fp8q_status launch_scatter_copy(const uint8_t* xq, const uint8_t* xsf, int64_t r
   if (blocks > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const cudaError_t rc = launch_after(scatter_copy_kernel, (unsigned)blocks, kSThreads, 0, stream,
                                       reinterpret_cast<const uint4*>(xq), xsf, rows, ncb, row_id_map, (int)slots,
-                                      reinterpret_cast<uint4*>(q), sf, scatter_ctas, pad_slots, offsets, totals);
+                                      reinterpret_cast<uint4*>(q), sf, scatter_ctas, pad_slots, offsets, totals,
+                                      max_rows);
   return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -554,9 +578,8 @@ fp8q_status launch_permute_pad_quant(const DeviceInfo& dev, const void* x, int64
                                      const int32_t* topk_idx, int32_t topk, int32_t num_experts, int32_t align,
                                      uint8_t* q, uint8_t* sf, int64_t max_out_rows, int32_t* expert_offsets,
                                      int32_t* row_id_map, void* workspace, cudaStream_t stream) {
-  (void)max_out_rows;
   return permute_pad(dev, x, nullptr, nullptr, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
-                     expert_offsets, row_id_map, workspace, stream);
+                     max_out_rows, expert_offsets, row_id_map, workspace, stream);
 }
 
 fp8q_status launch_permute_pad_fp8(const DeviceInfo& dev, const uint8_t* xq, const uint8_t* xsf, int64_t tokens,
@@ -564,9 +587,8 @@ fp8q_status launch_permute_pad_fp8(const DeviceInfo& dev, const uint8_t* xq, con
                                    int32_t align, uint8_t* q, uint8_t* sf, int64_t max_out_rows,
                                    int32_t* expert_offsets, int32_t* row_id_map, void* workspace,
                                    cudaStream_t stream) {
-  (void)max_out_rows;
   return permute_pad(dev, nullptr, xq, xsf, tokens, hidden, topk_idx, topk, num_experts, align, q, sf,
-                     expert_offsets, row_id_map, workspace, stream);
+                     max_out_rows, expert_offsets, row_id_map, workspace, stream);
 }
 
 }  // namespace fp8q

@@ -30,10 +30,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiles_kernel(const uint4* 
                                                                     uint8_t* __restrict__ sf, int64_t n_tiles,
                                                                     const int32_t* __restrict__ limit_rows,
                                                                     int64_t tiles_per_row) {
-  pdl_wait();
+  pdl_wait_for(x, limit_rows);
   pdl_trigger();
   if (limit_rows != nullptr) {
-    const int64_t lim = (int64_t)__ldg(limit_rows);
+    const int64_t lim = (int64_t)ld_g(limit_rows);
     n_tiles = lim <= 0 ? 0 : min(n_tiles, lim * tiles_per_row);
   }
   const int lane = threadIdx.x & 31;

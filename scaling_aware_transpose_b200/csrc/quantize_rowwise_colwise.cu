@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                                     uint8_t* __restrict__ sft) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
-  pdl_wait();
+  pdl_wait_for(x);
   pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;
@@ -69,8 +69,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int rl = p * 32 + rsub;
     if (kColwise || r0 + rl < rows) {
       const uint4* src = reinterpret_cast<const uint4*>(xb + rl * cols);
-      v0[p] = __ldg(src + sub);
-      v1[p] = __ldg(src + 8 + sub);
+      v0[p] = ld_g(src + sub);
+      v1[p] = ld_g(src + 8 + sub);
     } else {
       v0[p] = v1[p] = make_uint4(0u, 0u, 0u, 0u);
     }

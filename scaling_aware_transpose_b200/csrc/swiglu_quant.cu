@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) swiglu_quant_kernel(cons
   __shared__ __align__(16) uint8_t tile[128 * 128];
   __shared__ __align__(16) uint8_t e_row[128];
   __shared__ int e_max_sh;
-  pdl_wait();
+  pdl_wait_for(gate, up);
   pdl_trigger();
   const int tid = threadIdx.x;
   const int ncb = cols >> 7;

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
                                                                    const float* __restrict__ weights, int64_t tokens,
                                                                    int topk, uint16_t* __restrict__ out,
                                                                    int* status) {
-  pdl_wait();
+  pdl_wait_for(y, y_sf, row_id_map, weights);
   pdl_trigger();
   const int nch = hidden >> 4;
   const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -85,8 +85,8 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
       float wg[kK];
 #pragma unroll
       for (int s = 0; s < kK; ++s) {
-        rr[s] = __ldg(row_id_map + t * kK + s);
-        wg[s] = weights != nullptr ? __ldg(weights + t * kK + s) : 1.0f;
+        rr[s] = ld_g(row_id_map + t * kK + s);
+        wg[s] = weights != nullptr ? ld_g(weights + t * kK + s) : 1.0f;
       }
 #pragma unroll
       for (int s0 = 0; s0 < kK; s0 += kBatch) {
@@ -105,8 +105,8 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
               record_status(status, FP8Q_ERR_DEVICE);  // the slot is skipped
             } else {
               use[b] = true;
-              d[b] = __ldg(reinterpret_cast<const uint4*>(y + r * hidden + h0));
-              sc[b] = ue8m0_scale(__ldg(y_sf + r * ntile + (h0 >> 7)));
+              d[b] = ld_g(reinterpret_cast<const uint4*>(y + r * hidden + h0));
+              sc[b] = ue8m0_scale(ld_g(y_sf + r * ntile + (h0 >> 7)));
             }
           }
         }
@@ -136,19 +136,19 @@ __global__ void __launch_bounds__(kThreads) unpermute_unpad_kernel(const uint8_t
         sc[b] = 1.0f;
         d0[b] = d1[b] = make_uint4(0u, 0u, 0u, 0u);
         if (s < topk) {
-          const int64_t r = __ldg(row_id_map + t * topk + s);
+          const int64_t r = ld_g(row_id_map + t * topk + s);
           if (r < 0 || r >= rows) {
             record_status(status, FP8Q_ERR_DEVICE);  // the slot is skipped
           } else {
             use[b] = true;
-            if (weights != nullptr) ws[b] = __ldg(weights + t * topk + s);
+            if (weights != nullptr) ws[b] = ld_g(weights + t * topk + s);
             if (kFp8) {
-              d0[b] = __ldg(reinterpret_cast<const uint4*>(y + r * hidden + h0));
-              sc[b] = ue8m0_scale(__ldg(y_sf + r * ntile + (h0 >> 7)));
+              d0[b] = ld_g(reinterpret_cast<const uint4*>(y + r * hidden + h0));
+              sc[b] = ue8m0_scale(ld_g(y_sf + r * ntile + (h0 >> 7)));
             } else {
               const uint4* src = reinterpret_cast<const uint4*>(y + (r * hidden + h0) * 2);
-              d0[b] = __ldg(src);
-              d1[b] = __ldg(src + 1);
+              d0[b] = ld_g(src);
+              d1[b] = ld_g(src + 1);
             }
           }
         }
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) unpermute_fp8_ring(const uint
                                                                       int64_t tokens, uint16_t* __restrict__ out,
                                                                       int* status) {
   extern __shared__ __align__(128) uint8_t smem[];
-  pdl_wait();
+  pdl_wait_for(y, y_sf, row_id_map, weights);
   pdl_trigger();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // stage filled: 32 async arrivals + 1 expect-tx arrival
   uint64_t* empty = full + kRingStages;                 // stage released: one arrival per consumer warp
@@ -252,8 +252,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) unpermute_fp8_ring(const uint
     int32_t r_next = -1;
     float w_next = 1.0f;
     if (ntok > 0 && lane < kK) {
-      r_next = __ldg(row_id_map + (int64_t)blockIdx.x * kK + lane);
-      w_next = weights != nullptr ? __ldg(weights + (int64_t)blockIdx.x * kK + lane) : 1.0f;
+      r_next = ld_g(row_id_map + (int64_t)blockIdx.x * kK + lane);
+      w_next = weights != nullptr ? ld_g(weights + (int64_t)blockIdx.x * kK + lane) : 1.0f;
     }
     for (int64_t i = 0; i < ntok; ++i) {
       const int st = (int)(i % kRingStages);
@@ -261,8 +261,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) unpermute_fp8_ring(const uint
       const float w = w_next;
       if (i + 1 < ntok && lane < kK) {  // the next token's indices, in flight while this one is issued
         const int64_t tn = blockIdx.x + (i + 1) * gridDim.x;
-        r_next = __ldg(row_id_map + tn * kK + lane);
-        w_next = weights != nullptr ? __ldg(weights + tn * kK + lane) : 1.0f;
+        r_next = ld_g(row_id_map + tn * kK + lane);
+        w_next = weights != nullptr ? ld_g(weights + tn * kK + lane) : 1.0f;
       }
       if (i >= kRingStages &&
           !mbar_wait_bounded(&empty[st], (uint32_t)(((i / kRingStages) - 1) & 1), kWaitTimeoutNs)) {

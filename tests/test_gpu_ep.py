@@ -135,6 +135,66 @@ def test_ep_duplicate_experts_and_one_hot_rank():
             assert_bytes_equal(host(sf)[:n], osf[:n], f"{mode} rank {d} SF")
 
 
+def test_ep_back_to_back_calls_share_one_workspace():
+    """Two different routings, packed (and then receive-permuted) alternately on one stream
+    through ONE workspace, with no synchronisation between the calls.  The kernels of a
+    call may be placed before the previous call's kernels end (dependent launches), so a
+    kernel that read routing data written inside its own call before waiting for it would
+    see the other routing's stale values here.  Every result must still be the oracle's."""
+    W, T, H, K, Eloc, align = 4, 4096, 256, 8, 8, 128
+    xs, idx_a = _sources(W, T, H, K, Eloc, seed=21)
+    _, idx_b = _sources(W, T, H, K, Eloc, seed=77)
+    q0, sf0 = dev(xs[0][0]), dev(xs[0][1])
+    routings = [dev(idx_a[0]), dev(idx_b[0])]
+    cap = T * min(W, K)
+    ws = torch.empty(sat.fp8q_ep_pack_workspace_bytes(T, W), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in routings:
+        outs.append((torch.empty((cap, H), dtype=torch.uint8, device="cuda"),
+                     torch.empty((cap, H // 128), dtype=torch.uint8, device="cuda"),
+                     torch.empty((cap, K), dtype=torch.int32, device="cuda"),
+                     torch.empty((W + 1,), dtype=torch.int32, device="cuda"),
+                     torch.empty((T, W), dtype=torch.int32, device="cuda")))
+    for rep in range(6):
+        for r, idx in enumerate(routings):
+            o = outs[r]
+            sat.fp8q_ep_dispatch_pack(q0, sf0, T, H, idx, K, W, Eloc, o[0], o[1], o[2], cap, o[3], o[4], ws,
+                                      ws.numel())
+    device_status_ok()
+    wants = [oracle.ep_dispatch_pack(xs[0][0], xs[0][1], i, W, Eloc) for i in (idx_a[0], idx_b[0])]
+    for r in range(2):
+        _check_pack(outs[r], wants[r], T)
+    # the receive side: rank 0's segment of each routing's pack, alternately
+    segs = []
+    for r in range(2):
+        a, b = int(wants[r][3][0]), int(wants[r][3][1])
+        segs.append([(outs[r][0][a:b], outs[r][1][a:b], outs[r][2][a:b], b - a)])
+    rows = [sg[0][3] for sg in segs]
+    rws = torch.empty(max(sat.fp8q_ep_recv_workspace_bytes(n, K, Eloc) for n in rows), dtype=torch.uint8,
+                      device="cuda")
+    rout = []
+    for n in rows:
+        m = sat.permute_max_rows(n, K, Eloc, align)
+        rout.append((torch.empty((m, H), dtype=torch.uint8, device="cuda"),
+                     torch.empty((m, H // 128), dtype=torch.uint8, device="cuda"),
+                     torch.empty((Eloc + 1,), dtype=torch.int32, device="cuda"),
+                     torch.empty((max(n * K, 1),), dtype=torch.int32, device="cuda"), m))
+    for rep in range(6):
+        for r in range(2):
+            o = rout[r]
+            sat.fp8q_ep_recv_permute_fp8(segs[r], H, K, Eloc, align, o[0], o[1], o[4], o[2], o[3], rws, rws.numel())
+    device_status_ok()
+    for r in range(2):
+        a, b = int(wants[r][3][0]), int(wants[r][3][1])
+        oq, osf, ooff, ormap = oracle.ep_recv_permute(wants[r][0][a:b], wants[r][1][a:b], wants[r][2][a:b], Eloc,
+                                                      align)
+        assert_bytes_equal(host(rout[r][2]), ooff, f"routing {r} offsets")
+        n = int(ooff[-1])
+        assert_bytes_equal(host(rout[r][3])[:rows[r] * K], ormap, f"routing {r} row_id_map")
+        assert_bytes_equal(host(rout[r][0])[:n], oq[:n], f"routing {r} Q")
+        assert_bytes_equal(host(rout[r][1])[:n], osf[:n], f"routing {r} SF")
+
+
 def test_ep_bad_ids_set_device_status():
     q = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
     sf = torch.full((4, 1), 127, dtype=torch.uint8, device="cuda")
