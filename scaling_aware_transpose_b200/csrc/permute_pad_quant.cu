@@ -10,10 +10,12 @@
 //
 // Launches: (1) per-chunk expert histograms, (2) one CTA scans them into padded expert
 // offsets and per-chunk bases, (3) stable ranks within each chunk with __match_any_sync
-// (eight warps per chunk for up to 512 experts, one warp beyond), (4) the streaming
-// scatter-quantize over all (token, tile) pairs, whose trailing CTAs zero-fill the
-// padding rows.  (2)-(4) are programmatic dependent launches that overlap the tail of
-// their predecessor (see pdl_wait).  Workspace: counts[C][E], bases[C][E], totals[E].
+// (eight warps per chunk for up to 512 experts, one warp beyond; for small routings (2)
+// is folded into (3)), (4) the streaming scatter-quantize over all (token, tile) pairs,
+// whose trailing CTAs zero-fill the padding rows.  All are programmatic dependent
+// launches (see pdl_wait): (1) waits for the previous kernel in the stream before its
+// first access, (2)-(4) overlap their predecessor and wait only where they first read
+// its output.  Workspace: counts[C][E], bases[C][E], totals[E].
 // The FP8-input variant (the dispatch already delivered row-wise codes and scales) shares
 // (1)-(3) and the padding; its step (4) copies each token's codes and scale bytes to its
 // rows.
