@@ -97,6 +97,18 @@ def test_ep_many_ranks_and_empty_segments():
     run_ep(64, 20, 128, 2, 1, 16, seed=3)
 
 
+def test_ep_pack_large_routing_takes_the_unfused_rank_path():
+    """64 ranks x 4096 tokens: 262144 destination pairs, too many chunks for the fused rank
+    kernel, so the pack runs the routing's separate scan and rank launches."""
+    W, T, H, K, Eloc = 64, 4096, 128, 2, 1
+    xs, idx = _sources(1, T, H, K, W * Eloc, seed=6)
+    rng = np.random.default_rng(6)
+    idx = synthetic.zipf_topk(T, W * Eloc, K, rng)
+    got = sat.ep_dispatch_pack(dev(xs[0][0]), dev(xs[0][1]), dev(idx), W, Eloc)
+    device_status_ok()
+    _check_pack(got, oracle.ep_dispatch_pack(xs[0][0], xs[0][1], idx, W, Eloc), T)
+
+
 def test_ep_duplicate_experts_and_one_hot_rank():
     """Routing the Zipf sampler never draws: two slots of a token on the same expert (one
     send row, two slot ids, two expert rows), and every token routed to rank 2's experts
