@@ -70,9 +70,11 @@ def kernel_sources(kind: str):
             "unpermute": "unpermute_unpad.cu", "unpermute_fp8": "unpermute_unpad.cu", "mx32": "mx32.cu",
             "mx32_quantize": "mx32.cu", "direct_grouped": "direct_transpose.cu", "naive": "naive_transpose.cu",
             "direct_stress": "direct_transpose.cu",
-            "permute_fp8": "permute_pad_quant.cu", "ep_pack": "ep_dispatch.cu", "ep_recv": "ep_dispatch.cu"}[kind]
+            "permute_fp8": "permute_pad_quant.cu", "ep_pack": "ep_dispatch.cu", "ep_recv": "ep_dispatch.cu",
+            "permute_e512": "permute_pad_quant.cu", "permute_e4096": "permute_pad_quant.cu",
+            "unpermute_fp8_k": "unpermute_unpad.cu"}[kind]
     extra = ["permute_common.cuh", "permute_pad_quant.cu"] if kind in ("ep_pack", "ep_recv") else []
-    if kind in ("permute", "permute_fp8"):
+    if kind in ("permute", "permute_fp8", "permute_e512", "permute_e4096"):
         extra = ["permute_common.cuh"]
     return [os.path.join(csrc, main), os.path.join(csrc, "common.cuh")] + [os.path.join(csrc, e) for e in extra]
 
@@ -838,6 +840,23 @@ def run_profile(args):
         wts = torch.from_numpy(c["weights"]).cuda()
         calls = {"unpermute": lambda: sat.unpermute_unpad(y, rmap, K, wts),
                  "unpermute_fp8": lambda: sat.unpermute_unpad(pq, rmap, K, None, psf)}
+    elif args.profile in ("permute_e512", "permute_e4096"):
+        # routings too wide for the fused rank kernel: the chunk scan (a CTA per 32 experts)
+        # and the eight-warp rank, at 512 and at the 4096-expert maximum
+        E = 512 if args.profile == "permute_e512" else 4096
+        d = synthetic.moe(num_experts=E)
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        calls = {args.profile: lambda: sat.permute_pad_quant(x, idx, E, 16)}
+    elif args.profile == "unpermute_fp8_k":
+        # FP8 combine with hidden % 1024 != 0: the per-top-k kernel instead of the ring
+        d = synthetic.moe(hidden=7040)
+        x = synthetic.to_torch_bf16(d["x"]).cuda()
+        idx = torch.from_numpy(d["topk_idx"]).cuda()
+        K = idx.shape[1]
+        pq, psf, off, rmap = sat.permute_pad_quant(x, idx, d["num_experts"], 128)
+        del x
+        calls = {"unpermute_fp8_k": lambda: sat.unpermute_unpad(pq, rmap, K, None, psf)}
     else:  # permute
         d = synthetic.moe()
         x = synthetic.to_torch_bf16(d["x"]).cuda()
@@ -864,7 +883,8 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=1024, help="rows of the workload per reference step")
     ap.add_argument("--profile", choices=["quantize", "direct", "naive", "swiglu", "permute", "rowwise_colwise",
                                           "unpermute", "unpermute_fp8", "mx32", "permute_fp8", "mx32_quantize",
-                                          "direct_grouped", "ep_pack", "ep_recv", "direct_stress"],
+                                          "direct_grouped", "ep_pack", "ep_recv", "direct_stress", "permute_e512",
+                                          "permute_e4096", "unpermute_fp8_k"],
                     default=None,
                     help="launch only this kernel (for ncu captures); prints no bench line")
     args = ap.parse_args(argv)

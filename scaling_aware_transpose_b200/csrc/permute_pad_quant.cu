@@ -8,10 +8,11 @@
 // (t, s) row-major order; each expert segment is padded with zero rows (codes 0, scale
 // byte 127) to a multiple of `align`.
 //
-// Launches: (1) per-chunk expert histograms, (2) one CTA scans them into padded expert
-// offsets and per-chunk bases, (3) stable ranks within each chunk with __match_any_sync
-// (eight warps per chunk for up to 512 experts, one warp beyond; for small routings (2)
-// is folded into (3)), (4) the streaming scatter-quantize over all (token, tile) pairs,
+// Launches: (1) per-chunk expert histograms, (2) a CTA per 32 experts scans them over the
+// chunks into per-chunk bases and expert totals, (3) stable ranks within each chunk with
+// __match_any_sync, eight warps per chunk, each CTA scanning the padded totals into the
+// expert offsets itself (for small routings (2) is folded into (3)), (4) the streaming
+// scatter-quantize over all (token, tile) pairs,
 // whose trailing CTAs zero-fill the padding rows.  All are programmatic dependent
 // launches (see pdl_wait): (1) waits for the previous kernel in the stream before its
 // first access, (2)-(4) overlap their predecessor and wait only where they first read
@@ -26,19 +27,26 @@ namespace fp8q {
 namespace {
 
 // allow_drop: an id of -1 means "not routed here" (no row, no error); any other id
-// outside [0, E) records FP8Q_ERR_DEVICE.
+// outside [0, E) records FP8Q_ERR_DEVICE.  Launched with 256 threads.
 __global__ void __launch_bounds__(256) count_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
                                                     bool allow_drop, int32_t* __restrict__ counts, int* status) {
   extern __shared__ int32_t hist[];
   pdl_wait_for(idx);
   pdl_trigger();
+  const int64_t p0 = (int64_t)blockIdx.x * kChunk;
+  constexpr int kPer = kChunk / 256;
+  int32_t ids[kPer];  // this thread's ids, in flight while the histogram is cleared
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int64_t p = p0 + u * 256 + threadIdx.x;
+    ids[u] = p < npairs ? ld_g(idx + p) : -1;
+  }
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int64_t p0 = (int64_t)blockIdx.x * kChunk;
-  for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
-    const int64_t p = p0 + i;
-    if (p >= npairs) break;
-    const int32_t e = ld_g(idx + p);
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    if (p0 + u * 256 + threadIdx.x >= npairs) break;
+    const int32_t e = ids[u];
     if (e < 0 || e >= E) {
       if (!(allow_drop && e == -1)) record_status(status, FP8Q_ERR_DEVICE);
       continue;
@@ -59,131 +67,103 @@ __device__ __forceinline__ int32_t warp_incl_scan32(int32_t v, int lane) {
   return v;
 }
 
-// One CTA of 1024 threads (32 warps); totals and offsets stay in shared memory, so the
-// kernel is a short chain: (1) warp w sums expert e's counts over the chunks (e = w,
-// w + 32, ...; eight loads in flight per lane) -> totals; (2) exclusive scan of the padded
-// sizes ceil(total/align)*align over the experts (per-thread runs, a warp scan and a scan
-// of the 32 warp sums) -> offsets; (3) warp per expert again: exclusive scan over the
-// chunks -> bases[c][e].  Every value fits in int32: the host caps the padded row count
-// below 2^31.
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int64_t C, int E, int align,
-                                                    int32_t* __restrict__ offsets, int32_t* __restrict__ bases,
-                                                    int32_t* __restrict__ totals) {
-  __shared__ int32_t s_tot[kMaxExperts];
-  __shared__ int32_t s_off[kMaxExperts];
-  __shared__ int32_t s_warp[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Per-expert prefix over the chunks, for routings too large for the fused rank kernel.
+// CTA b owns experts 32b..32b+31 with one lane per expert, so each chunk's 32 counts are
+// one 128-byte load; its 32 warps split the chunks into contiguous ranges.  Each lane sums
+// its range, the ranges' sums are scanned across the warps in shared memory, and each lane
+// then walks its range again writing bases[c][e] = the pairs of expert e in chunks before
+// c.  Warp 0 writes totals[e].  The padded offsets are left to the rank kernel, whose CTAs
+// each scan the E totals themselves (no cross-CTA step here).
+__global__ void __launch_bounds__(1024) chunk_scan_kernel(const int32_t* __restrict__ counts, int64_t C, int E,
+                                                          int32_t* __restrict__ bases, int32_t* __restrict__ totals) {
+  __shared__ int32_t s_part[32][32];  // [warp][lane]: the warp's range sum for the lane's expert
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const bool live = e < E;
+  const int64_t per = (C + 31) / 32;
+  const int64_t c0 = min(C, w * per), c1 = min(C, c0 + per);
   pdl_trigger();
   pdl_wait_for(counts);  // the histograms
-  for (int e = warp; e < E; e += 32) {
-    int32_t acc = 0;
-    for (int64_t c0 = 0; c0 < C; c0 += 8 * 32) {
-      int32_t v[8];
+  int32_t sum = 0;
+  for (int64_t c = c0; c < c1; c += 8) {
+    int32_t v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t c = c0 + u * 32 + lane;
-        v[u] = c < C ? ld_g(counts + c * E + e) : 0;
-      }
+    for (int u = 0; u < 8; ++u) v[u] = live && c + u < c1 ? ld_g(counts + (c + u) * E + e) : 0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc += v[u];
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if (lane == 0) {
-      s_tot[e] = acc;
-      totals[e] = acc;
-    }
+    for (int u = 0; u < 8; ++u) sum += v[u];
   }
+  s_part[w][lane] = sum;
   __syncthreads();
-  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;  // experts per thread
-  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-  int32_t local = 0;
-  for (int e = e0; e < e1; ++e) local += (s_tot[e] + align - 1) / align * align;
-  const int32_t incl = warp_incl_scan32(local, lane);
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int32_t w = s_warp[lane];
-    s_warp[lane] = warp_incl_scan32(w, lane) - w;  // exclusive prefix of the warp sums
+  int32_t run = 0, tot = 0;
+#pragma unroll 8
+  for (int ww = 0; ww < 32; ++ww) {
+    const int32_t v = s_part[ww][lane];
+    run += ww < w ? v : 0;
+    tot += v;
   }
-  __syncthreads();
-  int32_t run = s_warp[warp] + incl - local;
-  for (int e = e0; e < e1; ++e) {
-    s_off[e] = run;
-    offsets[e] = run;
-    run += (s_tot[e] + align - 1) / align * align;
-  }
-  if (tid == (int)blockDim.x - 1) offsets[E] = run;  // threads past the last expert hold the total
-  __syncthreads();
-  for (int e = warp; e < E; e += 32) {
-    int32_t carry = s_off[e];
-    for (int64_t c0 = 0; c0 < C; c0 += 8 * 32) {
-      int32_t v[8];
+  if (w == 0 && live) totals[e] = tot;
+  for (int64_t c = c0; c < c1; c += 8) {
+    int32_t v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t c = c0 + u * 32 + lane;
-        v[u] = c < C ? ld_g(counts + c * E + e) : 0;
-      }
+    for (int u = 0; u < 8; ++u) v[u] = live && c + u < c1 ? ld_g(counts + (c + u) * E + e) : 0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t c = c0 + u * 32 + lane;
-        const int32_t inc = warp_incl_scan32(v[u], lane);
-        if (c < C) bases[c * E + e] = carry + inc - v[u];
-        carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
-      }
+    for (int u = 0; u < 8; ++u) {
+      if (live && c + u < c1) bases[(c + u) * E + e] = run;
+      run += v[u];
     }
   }
 }
 
-__global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ idx, int64_t npairs, int E,
-                                                  const int32_t* __restrict__ bases, int32_t* __restrict__ row_id_map,
-                                                  bool ids_wait) {
-  extern __shared__ int32_t run[];
-  const int lane = threadIdx.x;
-  const int64_t p0 = (int64_t)blockIdx.x * kChunk;
-  int32_t ids[kChunk / 32];
-  if (ids_wait) pdl_wait_for(idx);  // the ids were written inside this call (see route_ranks)
+// Exclusive scan of the padded group sizes ceil(s[e]/align)*align over the groups by the
+// whole CTA, in place: s[e] holds group e's total on entry and its offset on return.  Warp
+// w takes the w-th contiguous segment of the groups: it sums the segment (lanes striding),
+// the warps' sums are scanned through s_wsum (one word per warp), and the warp walks its
+// segment again 32 groups per step (lane = group, so shared accesses are conflict-free)
+// with a warp scan and a carry.  offsets != nullptr also stores offsets[0..E].  Ends with
+// a barrier.
+__device__ __forceinline__ void block_pad_offsets(int32_t* s, int32_t* s_wsum, int E, int align,
+                                                  int32_t* __restrict__ offsets) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int seg = (E + nw - 1) / nw;
+  const int e0 = min(E, w * seg), e1 = min(E, e0 + seg);
+  int32_t acc = 0;
+  for (int e = e0 + lane; e < e1; e += 32) acc += (s[e] + align - 1) / align * align;
 #pragma unroll
-  for (int i = 0; i < kChunk / 32; ++i) {
-    const int64_t p = p0 + i * 32 + lane;
-    ids[i] = p < npairs ? ld_g(idx + p) : -1;
-  }
-  pdl_trigger();
-  pdl_wait_for(bases);  // the bases
-  for (int e = lane; e < E; e += 32) run[e] = bases[(int64_t)blockIdx.x * E + e];
-  __syncwarp();
-#pragma unroll 4
-  for (int i = 0; i < kChunk / 32; ++i) {
-    const int64_t p = p0 + i * 32 + lane;
-    const bool live = p < npairs;
-    const int32_t e = ids[i];
-    const bool ok = live && e >= 0 && e < E;
-    const int32_t key = ok ? e : -1 - lane;  // invalid lanes never match anyone
-    const unsigned same = __match_any_sync(0xFFFFFFFFu, key);
-    const int rank = __popc(same & ((1u << lane) - 1u));
-    const int base = ok ? run[e] : 0;
-    __syncwarp();
-    if (ok) {
-      row_id_map[p] = base + rank;
-      if (rank == 0) run[e] = base + __popc(same);
-    } else if (live) {
-      row_id_map[p] = -1;
+  for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (lane == 0) s_wsum[w] = acc;
+  __syncthreads();
+  int32_t run = 0;
+  for (int ww = 0; ww < w; ++ww) run += s_wsum[ww];
+  for (int eb = e0; eb < e1; eb += 32) {
+    const int e = eb + lane;
+    const int32_t padded = e < e1 ? (s[e] + align - 1) / align * align : 0;
+    const int32_t incl = warp_incl_scan32(padded, lane);
+    if (e < e1) {
+      s[e] = run + incl - padded;
+      if (offsets) offsets[e] = run + incl - padded;
     }
-    __syncwarp();
+    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
   }
+  if (offsets && w == nw - 1 && lane == 0) offsets[E] = run;  // past every segment: the grand total
+  __syncthreads();
 }
 
-// Rank with 8 warps per chunk, for E <= kRankMultiMaxE (per-warp counts in shared
+// Rank with 8 warps per chunk, after chunk_scan_kernel (per-warp counts in shared
 // memory): warp w owns pairs 128w..128w+127 of the chunk.  (A) each warp counts its pairs
-// per expert; (B) per expert, an exclusive prefix over the warps on top of the chunk's
-// base; (C) each warp ranks its pairs from its own bases.  Same stable (t, s) order as
-// rank_kernel with 8 serial steps per warp instead of 32.
+// per expert; (B) the CTA scans the padded expert totals into offsets (CTA 0 stores them)
+// and, per expert, takes an exclusive prefix over the warps on top of offset + the chunk's
+// base; (C) each warp ranks its pairs from its own bases, 8 serial steps per warp.  Stable
+// (t, s) order.  Shared memory: 9E + 8 words (147 KB at 4096 experts, one CTA per SM).
 constexpr int kRankWarps = 8;
-constexpr int kRankMultiMaxE = 512;
+inline size_t rank_multi_smem(int E) { return ((size_t)(kRankWarps + 1) * E + kRankWarps) * sizeof(int32_t); }
 __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32_t* __restrict__ idx, int64_t npairs,
-                                                                     int E, const int32_t* __restrict__ bases,
+                                                                     int E, int align, const int32_t* __restrict__ bases,
+                                                                     const int32_t* __restrict__ totals,
+                                                                     int32_t* __restrict__ offsets,
                                                                      int32_t* __restrict__ row_id_map, bool ids_wait) {
-  extern __shared__ int32_t s_cnt[];  // [kRankWarps][E]
+  extern __shared__ int32_t s_cnt[];  // [kRankWarps][E] | off[E] | warp sums[kRankWarps]
+  int32_t* s_off = s_cnt + kRankWarps * E;
+  int32_t* s_wsum = s_off + E;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   constexpr int kPer = kChunk / kRankWarps / 32;  // iterations per warp
   const int64_t p0 = (int64_t)blockIdx.x * kChunk + w * (kChunk / kRankWarps);
@@ -207,15 +187,35 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
     if (ok && lane == __ffs(same) - 1) mine[e] += __popc(same);
     __syncwarp();
   }
-  __syncthreads();
-  pdl_wait_for(bases);  // the bases
-  for (int e = tid; e < E; e += blockDim.x) {
-    int32_t run = bases[(int64_t)blockIdx.x * E + e];
+  pdl_wait_for(bases, totals);  // the chunk bases and expert totals
+  // eight loads in flight per thread in both passes (E up to 4096: 16 per thread)
+  constexpr int kB = 8, kT = kRankWarps * 32;
+  for (int eb = tid; eb < E; eb += kB * kT) {
+    int32_t v[kB];
 #pragma unroll
-    for (int ww = 0; ww < kRankWarps; ++ww) {
-      const int32_t v = s_cnt[ww * E + e];
-      s_cnt[ww * E + e] = run;
-      run += v;
+    for (int u = 0; u < kB; ++u) v[u] = eb + u * kT < E ? ld_g(totals + eb + u * kT) : 0;
+#pragma unroll
+    for (int u = 0; u < kB; ++u)
+      if (eb + u * kT < E) s_off[eb + u * kT] = v[u];
+  }
+  __syncthreads();
+  block_pad_offsets(s_off, s_wsum, E, align, blockIdx.x == 0 ? offsets : nullptr);
+  const int32_t* my_bases = bases + (int64_t)blockIdx.x * E;
+  for (int eb = tid; eb < E; eb += kB * kT) {
+    int32_t b[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) b[u] = eb + u * kT < E ? ld_g(my_bases + eb + u * kT) : 0;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int e = eb + u * kT;
+      if (e >= E) break;
+      int32_t run = s_off[e] + b[u];
+#pragma unroll
+      for (int ww = 0; ww < kRankWarps; ++ww) {
+        const int32_t c = s_cnt[ww * E + e];
+        s_cnt[ww * E + e] = run;
+        run += c;
+      }
     }
   }
   __syncthreads();
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_multi_kernel(const int32
 
 // Rank with the scan folded in, for small routings (see route_pairs): the same stable
 // ranking as rank_multi_kernel, but each CTA derives its own bases from the per-chunk
-// histograms instead of reading them from scan_kernel.  A warp per group sums the group's
+// histograms instead of reading them from chunk_scan_kernel.  A warp per group sums the group's
 // counts over all chunks (its total) and over the chunks before this one (this chunk's
 // prefix), lanes striding over the chunks; an exclusive scan of the padded totals over the
 // groups gives the offsets.  CTA 0 also writes offsets[0..E] and the totals, which the
@@ -251,11 +251,10 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_fused_kernel(const int32
                                                                      int64_t C, int32_t* __restrict__ offsets,
                                                                      int32_t* __restrict__ totals,
                                                                      int32_t* __restrict__ row_id_map, bool ids_wait) {
-  extern __shared__ int32_t s_cnt[];  // [kRankWarps][E] | pre[E] | tot[E] | off[E] | warp sums[kRankWarps]
+  extern __shared__ int32_t s_cnt[];  // [kRankWarps][E] | pre[E] | tot[E] | warp sums[kRankWarps]
   int32_t* s_pre = s_cnt + kRankWarps * E;
   int32_t* s_tot = s_pre + E;
-  int32_t* s_off = s_tot + E;
-  int32_t* s_wsum = s_off + E;
+  int32_t* s_wsum = s_tot + E;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   constexpr int kPer = kChunk / kRankWarps / 32;
   const int64_t p0 = (int64_t)blockIdx.x * kChunk + w * (kChunk / kRankWarps);
@@ -280,47 +279,48 @@ __global__ void __launch_bounds__(kRankWarps * 32) rank_fused_kernel(const int32
     __syncwarp();
   }
   pdl_wait_for(counts);  // the histograms
-  for (int e = w; e < E; e += kRankWarps) {
-    int32_t tot = 0, pre = 0;
-    for (int64_t c = lane; c < C; c += 32) {
-      const int32_t v = ld_g(counts + c * E + e);
-      tot += v;
-      pre += c < (int64_t)blockIdx.x ? v : 0;
+  // warp w: groups w, w + 8, ... two at a time; lanes stride over the chunks, four strides
+  // at a time, so eight count loads are in flight per lane
+  for (int e0 = w; e0 < E; e0 += 2 * kRankWarps) {
+    int32_t tot[2] = {0, 0}, pre[2] = {0, 0};
+    for (int64_t c0 = lane; c0 < C; c0 += 4 * 32) {
+      int32_t v[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + j * kRankWarps;
+          const int64_t c = c0 + u * 32;
+          v[j][u] = e < E && c < C ? ld_g(counts + c * E + e) : 0;
+        }
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          tot[j] += v[j][u];
+          pre[j] += c0 + u * 32 < (int64_t)blockIdx.x ? v[j][u] : 0;
+        }
     }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
-      pre += __shfl_xor_sync(0xFFFFFFFFu, pre, o);
-    }
-    if (lane == 0) {
-      s_tot[e] = tot;
-      s_pre[e] = pre;
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        tot[j] += __shfl_xor_sync(0xFFFFFFFFu, tot[j], o);
+        pre[j] += __shfl_xor_sync(0xFFFFFFFFu, pre[j], o);
+      }
+      const int e = e0 + j * kRankWarps;
+      if (lane == 0 && e < E) {
+        s_tot[e] = tot[j];
+        s_pre[e] = pre[j];
+      }
     }
   }
   __syncthreads();
-  // exclusive scan of the padded totals over the groups (E <= 512: two per thread)
-  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
-  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-  int32_t local = 0;
-  for (int e = e0; e < e1; ++e) local += (s_tot[e] + align - 1) / align * align;
-  const int32_t incl = warp_incl_scan32(local, lane);
-  if (lane == 31) s_wsum[w] = incl;
-  __syncthreads();
-  int32_t wbase = 0;
-  for (int ww = 0; ww < w; ++ww) wbase += s_wsum[ww];
-  int32_t run = wbase + incl - local;
-  for (int e = e0; e < e1; ++e) {
-    s_off[e] = run;
-    if (blockIdx.x == 0) {
-      offsets[e] = run;
-      totals[e] = s_tot[e];
-    }
-    run += (s_tot[e] + align - 1) / align * align;
-  }
-  if (blockIdx.x == 0 && tid == (int)blockDim.x - 1) offsets[E] = run;  // the last thread holds the total
-  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int e = tid; e < E; e += blockDim.x) totals[e] = s_tot[e];
+  block_pad_offsets(s_tot, s_wsum, E, align, blockIdx.x == 0 ? offsets : nullptr);  // s_tot now holds offsets
   for (int e = tid; e < E; e += blockDim.x) {
-    int32_t r = s_off[e] + s_pre[e];
+    int32_t r = s_tot[e] + s_pre[e];
 #pragma unroll
     for (int ww = 0; ww < kRankWarps; ++ww) {
       const int32_t v = s_cnt[ww * E + e];
@@ -494,26 +494,26 @@ fp8q_status route_ranks(const DeviceInfo& dev, int64_t rows, const int32_t* idx,
   int32_t* counts = static_cast<int32_t*>(workspace);
   int32_t* bases = counts + C * E;
   int32_t* totals = bases + C * E;
-  const size_t hist_smem = (size_t)E * sizeof(int32_t);
   // Small routings (at most 32 count loads per lane in the fused kernel's reduction) fold
-  // the one-CTA scan into the rank kernel: one dependent launch fewer.
-  if (E <= kRankMultiMaxE && (int64_t)((E + kRankWarps - 1) / kRankWarps) * ((C + 31) / 32) <= 32) {
-    const size_t smem = ((size_t)(kRankWarps + 3) * E + kRankWarps) * sizeof(int32_t);
+  // the chunk scan into the rank kernel: one dependent launch fewer.
+  if (E <= 512 && (int64_t)((E + kRankWarps - 1) / kRankWarps) * ((C + 31) / 32) <= 32) {
+    const size_t smem = ((size_t)(kRankWarps + 2) * E + kRankWarps) * sizeof(int32_t);
     return launch_after(rank_fused_kernel, (unsigned)C, kRankWarps * 32, smem, stream, idx, npairs, E, (int)align,
                         (const int32_t*)counts, C, offsets, totals, row_id_map, ids_wait) == cudaSuccess
                ? FP8Q_OK
                : FP8Q_ERR_CUDA;
   }
-  if (launch_after(scan_kernel, 1, 1024, 0, stream, (const int32_t*)counts, C, E, (int)align, offsets, bases,
+  if (launch_after(chunk_scan_kernel, (unsigned)((E + 31) / 32), 1024, 0, stream, (const int32_t*)counts, C, E, bases,
                    totals) != cudaSuccess)
     return FP8Q_ERR_CUDA;
-  const cudaError_t rc =
-      E <= kRankMultiMaxE
-          ? launch_after(rank_multi_kernel, (unsigned)C, kRankWarps * 32, (size_t)kRankWarps * E * sizeof(int32_t),
-                         stream, idx, npairs, E, (const int32_t*)bases, row_id_map, ids_wait)
-          : launch_after(rank_kernel, (unsigned)C, 32, hist_smem, stream, idx, npairs, E, (const int32_t*)bases,
-                         row_id_map, ids_wait);
-  return rc == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  const size_t smem = rank_multi_smem(E);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(rank_multi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  return launch_after(rank_multi_kernel, (unsigned)C, kRankWarps * 32, smem, stream, idx, npairs, E, (int)align,
+                      (const int32_t*)bases, (const int32_t*)totals, offsets, row_id_map, ids_wait) == cudaSuccess
+             ? FP8Q_OK
+             : FP8Q_ERR_CUDA;
 }
 
 const int32_t* route_totals(const void* workspace, int64_t rows, int32_t slots, int32_t E) {

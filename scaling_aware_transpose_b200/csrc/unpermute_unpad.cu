@@ -21,11 +21,12 @@
 // takes as long to arrive as the index it depends on, so this saves a round trip per four
 // slots.  BF16 rows keep the index loads inside each batch, which measured faster there.
 //
-// FP8 rows with top-k <= 8 and hidden % 1024 == 0 take a warp-specialised ring instead
+// FP8 rows with top-k <= 8 and hidden % 512 == 0 take a warp-specialised ring instead
 // (unpermute_fp8_ring): one CTA per SM walks its tokens (blockIdx.x, + gridDim.x, ...)
 // through three shared-memory stages.  A producer warp keeps the next token's row
 // indices and weights in flight while it fills a stage: the token's K rows of codes
-// arrive by bulk copies (7 KB each at hidden 7168), its scale bytes by 8-byte cp.async,
+// arrive by bulk copies (7 KB each at hidden 7168), its scale bytes by 8-byte cp.async
+// (4-byte where hidden % 1024 != 0: the rows' scale bytes start 4-byte aligned there),
 // both tracked by the stage's mbarrier; the consumer warps dequantize and accumulate from
 // shared memory in the same slot order as above (identical bytes) and release the stage
 // through a second mbarrier.  Row loads no longer wait on the index loads, and three
@@ -283,17 +284,24 @@ __global__ void __launch_bounds__(kRingThreads, 1) unpermute_fp8_ring(const uint
         wsel[lane] = w;
       }
       const unsigned valid = __ballot_sync(0xFFFFFFFFu, lane < kK && r >= 0);
-      // scale rows in 8-byte pieces (hidden % 1024 == 0), spread over the lanes; every lane
-      // runs the same trip count so that the shuffle sees the whole warp
-      const int per_row = ntile >> 3;
+      // scale rows in 8-byte pieces (hidden % 1024 == 0) or 4-byte pieces (hidden % 512 ==
+      // 0), spread over the lanes; every lane runs the same trip count so that the shuffle
+      // sees the whole warp
+      const bool wide = (ntile & 7) == 0;
+      const int piece_bytes = wide ? 8 : 4;
+      const int per_row = ntile / piece_bytes;
       for (int idx0 = 0; idx0 < kK * per_row; idx0 += 32) {
         const int idx = idx0 + lane;
         const int k = min(idx / per_row, kK - 1), piece = idx - k * per_row;
         const int32_t rk = __shfl_sync(0xFFFFFFFFu, r, k);
-        if (idx < kK * per_row && rk >= 0)
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(scales + k * ntile + 8 * piece)),
-                       "l"(y_sf + (int64_t)rk * ntile + 8 * piece)
-                       : "memory");
+        if (idx < kK * per_row && rk >= 0) {
+          const uint32_t dst = smem_u32(scales + k * ntile + piece_bytes * piece);
+          const uint8_t* src = y_sf + (int64_t)rk * ntile + piece_bytes * piece;
+          if (wide)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+          else
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+        }
       }
       // this lane's arrival fires when its cp.asyncs have landed
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[st])) : "memory");
@@ -402,8 +410,10 @@ fp8q_status launch_unpermute_unpad(const DeviceInfo& dev, const void* y, const u
   const UnpermuteArgs a{static_cast<const uint8_t*>(y), y_sf, rows, (int)hidden, row_id_map, weights, tokens, topk,
                         static_cast<uint16_t*>(out), dev.status};
   const int ring_smem = 128 + kRingStages * ring_stage_bytes(topk, (int)hidden);
-  if (y_sf != nullptr && topk >= 1 && topk <= 8 && hidden % 1024 == 0 && ring_smem <= dev.max_smem_optin &&
-      (reinterpret_cast<uintptr_t>(y_sf) & 7u) == 0 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0) {
+  // the scale rows' copy pieces: 8 bytes when hidden % 1024 == 0, else 4 (hidden % 512 == 0)
+  const uintptr_t sf_align = hidden % 1024 == 0 ? 7u : 3u;
+  if (y_sf != nullptr && topk >= 1 && topk <= 8 && hidden % 512 == 0 && ring_smem <= dev.max_smem_optin &&
+      (reinterpret_cast<uintptr_t>(y_sf) & sf_align) == 0 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0) {
     const int grid = (int)(tokens < dev.num_sms ? tokens : dev.num_sms);
     cudaError_t e = cudaSuccess;
     switch (topk) {

@@ -4,6 +4,7 @@ arm's JSON line."""
 import json
 import multiprocessing as mp
 import os
+import re
 import socket
 
 import pytest
@@ -94,9 +95,18 @@ def test_reference_arm_other_ranks_do_nothing(capsys, monkeypatch):
 
 
 def test_every_profile_choice_names_existing_sources():
-    """Each --profile choice that has a summary under profiles/ maps to kernel sources that
-    exist, so a summary's source hash can always be recomputed."""
-    for kind in ("quantize", "direct", "swiglu", "permute", "rowwise_colwise", "unpermute", "unpermute_fp8", "mx32"):
+    """The --profile kind in each summary's command maps to kernel sources that exist, so
+    the summary's source hash can always be recomputed."""
+    d = os.path.join(bench.ROOT, "profiles")
+    kinds = set()
+    for name in sorted(os.listdir(d)):
+        if name.startswith("launches_"):
+            continue
+        m = re.search(r"--profile (\w+)", open(os.path.join(d, name)).read())
+        assert m, name
+        kinds.add(m.group(1))
+    assert {"permute_e512", "permute_e4096", "unpermute_fp8_k", "ep_pack", "ep_recv"} <= kinds
+    for kind in kinds:
         paths = bench.kernel_sources(kind)
         assert paths and all(os.path.exists(p) for p in paths), kind
     assert bench.kernel_sources("unpermute_fp8") == bench.kernel_sources("unpermute")

@@ -184,10 +184,28 @@ def test_permute_fp8_bad_index_sets_device_status():
 
 @pytest.mark.parametrize("tokens,E,K", [(700, 300, 4), (2500, 512, 2), (1800, 513, 3), (600, 4096, 8)])
 def test_permute_many_experts(tokens, E, K):
-    """Routing with many experts: the eight-warp rank path up to 512 experts, the one-warp
-    path beyond (513 and the 4096 maximum), uniform routing so most experts are hit."""
+    """Routing with many experts, too wide for the fused rank kernel: the per-32-expert
+    chunk scan and the eight-warp rank, with expert counts that are not multiples of 32
+    (300, 513) and the 4096 maximum (one rank CTA per SM), uniform routing so most experts
+    are hit."""
     rng = np.random.default_rng(E)
     idx = np.argsort(rng.random((tokens, E)), axis=1)[:, :K].astype(np.int32)
     d = {"x": synthetic.scaled_normal(tokens, 128, seed=E), "topk_idx": np.ascontiguousarray(idx)}
     check_permute(d, E, 16)
     check_permute_fp8(d["x"], d["topk_idx"], E, 16)
+
+
+@pytest.mark.parametrize("tokens,E,K", [(40000, 256, 8), (16384, 4096, 8), (70000, 33, 8)])
+def test_permute_wide_routing_many_chunks(tokens, E, K):
+    """Hundreds of 1024-pair chunks: each warp of the chunk scan walks a range of several
+    chunks in steps of eight with a ragged last step (313, 128 and 547 chunks), across
+    expert blocks with a partial last block (33 experts).  The 256-expert case is the full
+    top-8 routing of a 256-expert model; ids need not be distinct within a token."""
+    rng = np.random.default_rng(tokens + E)
+    if E <= 256:
+        idx = np.argsort(rng.random((tokens, E)), axis=1)[:, :K].astype(np.int32)
+    else:
+        idx = rng.integers(0, E, (tokens, K), dtype=np.int32)
+    d = {"x": synthetic.scaled_normal(tokens, 128, seed=E + 1), "topk_idx": np.ascontiguousarray(idx)}
+    check_permute(d, E, 16)
+    check_permute_fp8(d["x"], d["topk_idx"], E, 128)
