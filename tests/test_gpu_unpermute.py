@@ -42,12 +42,14 @@ def test_matches_oracle(fp8, weighted, T, H, K):
 @pytest.mark.parametrize("weighted", [False, True])
 @pytest.mark.parametrize("T,H,K", [(300, 1024, 1), (149, 1024, 2), (1000, 2048, 3), (5, 1024, 5), (777, 3072, 7),
                                    (2000, 8192, 8), (160, 7168, 4), (148, 1024, 6), (600, 3584, 8), (149, 1536, 3),
-                                   (77, 512, 1), (300, 2560, 6), (1000, 512, 8)])
+                                   (77, 512, 1), (300, 2560, 6), (1000, 512, 8), (5000, 1024, 2), (3000, 1536, 8),
+                                   (2000, 3584, 5)])
 def test_fp8_ring_matches_oracle(weighted, T, H, K):
     """FP8 rows with top-k <= 8 and hidden % 512 == 0 take the bulk-copy ring: fewer
-    tokens than SMs, exactly one per SM, and many tokens per CTA (the three stages wrap
-    around many times), every k, hidden up to 8192; the scale rows go in 8-byte pieces
-    when hidden % 1024 == 0 and in 4-byte pieces otherwise (512, 1536, 2560, 3584)."""
+    tokens than SMs, exactly one per SM, and many tokens per CTA (the stages wrap
+    around many times: up to 34 tokens per CTA at 5000 tokens),
+    every k, hidden up to 8192; the scale rows go in 8-byte pieces when hidden % 1024 ==
+    0 and in 4-byte pieces otherwise (512, 1536, 2560, 3584)."""
     R = T * K + 50
     y, sf, rmap, w = case(T, H, K, R, seed=3 * T + H + K, fp8=True)
     w = w if weighted else None
