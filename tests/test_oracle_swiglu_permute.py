@@ -153,25 +153,46 @@ def test_permute_brute_force_tiny(align):
     assert np.all(q[n:] == 0xEE) and np.all(sf[n:] == 0xEE)
 
 
-def test_permute_invariants_zipf():
-    d = synthetic.moe(tokens=512, hidden=256, num_experts=32, topk=8, seed=13)
-    align = 128
-    q, sf, off, rmap = oracle.permute_pad_quant(d["x"], d["topk_idx"], 32, align)
-    idx = d["topk_idx"]
-    counts = np.bincount(idx.ravel(), minlength=32)
-    assert counts.sum() == 512 * 8
+def _check_permute_invariants(x, idx, E, align):
+    """What the permute's definition fixes, checked without re-deriving it: each expert's
+    segment is its pair count rounded up to `align`, the offsets are their exclusive scan,
+    every pair has its own row inside its expert's segment, rows within a segment follow
+    (token, slot) order with no gap, every row holds its token's codes and scales, and the
+    padding rows are zero codes with scale byte 127."""
+    T, K = idx.shape
+    q, sf, off, rmap = oracle.permute_pad_quant(x, idx, E, align)
+    counts = np.bincount(idx.ravel(), minlength=E)
+    assert counts.sum() == T * K
     sizes = np.diff(off)
-    assert np.all(sizes % align == 0) and np.all(sizes >= counts) and np.all(sizes - counts < align)
+    assert off[0] == 0 and np.all(sizes % align == 0) and np.all(sizes >= counts) and np.all(sizes - counts < align)
+    assert np.array_equal(sizes == 0, counts == 0)
     assert len(np.unique(rmap)) == rmap.size
     e_of = idx.ravel()
     assert np.all((rmap >= off[e_of]) & (rmap < off[e_of] + counts[e_of]))
     # stable order: within an expert the rows follow (token, slot) order
-    for e in range(32):
-        r = rmap[e_of == e]
-        assert np.all(np.diff(r) == 1)
-    qx, sfx = oracle.quantize_rowwise(d["x"])
-    assert np.array_equal(q[rmap], np.repeat(qx, 8, axis=0))
-    assert np.array_equal(sf[rmap], np.repeat(sfx, 8, axis=0))
+    order = np.argsort(e_of, kind="stable")
+    assert np.array_equal(rmap[order], np.concatenate([np.arange(off[e], off[e] + counts[e]) for e in range(E)]))
+    qx, sfx = oracle.quantize_rowwise(x)
+    assert np.array_equal(q[rmap], np.repeat(qx, K, axis=0))
+    assert np.array_equal(sf[rmap], np.repeat(sfx, K, axis=0))
+    pad = np.ones(off[-1], bool)
+    pad[rmap] = False
+    assert np.all(q[:off[-1]][pad] == 0) and np.all(sf[:off[-1]][pad] == 127)
+
+
+def test_permute_invariants_zipf():
+    d = synthetic.moe(tokens=512, hidden=256, num_experts=32, topk=8, seed=13)
+    _check_permute_invariants(d["x"], d["topk_idx"], 32, 128)
+
+
+@pytest.mark.parametrize("T,E,K,align", [(2048, 4096, 8, 16), (3000, 513, 3, 1), (1500, 256, 8, 128)])
+def test_permute_invariants_wide_routing(T, E, K, align):
+    """Routings as wide as the library accepts (4096 experts, most of them empty), expert
+    counts that are not multiples of 32, ids repeated within a token."""
+    rng = np.random.default_rng(T + E)
+    idx = rng.integers(0, E, (T, K), dtype=np.int32)
+    idx[::5, 1] = idx[::5, 0]  # the same expert twice in one token
+    _check_permute_invariants(synthetic.scaled_normal(T, 128, seed=E), idx, E, align)
 
 
 def test_permute_rejects_bad_index():
